@@ -1,0 +1,162 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention forward.
+ *
+ * The forward of DSA as the DeepSeek-V3.2-Exp technical report defines it
+ * (Chinese translation on m.163.com, §1 "Architecture"):
+ *   1. lightning indexer  I_{t,s} = sum_j w_{t,j} * ReLU(q^I_{t,j} . k^I_s)   (Eq. 1)
+ *      over the H^I = 64 indexer heads, keys s <= pos(t) (causal);
+ *   2. fine-grained token selection S_t = Top-k(I_{t,:}), k <= 2048        (§1, §2.1)
+ *   3. sparse MLA in MQA mode: every one of the 128 query heads attends over
+ *      the selected shared latent rows c_s (576-d key = 512 latent + 64 rope,
+ *      value = first 512 dims), u_t = Attn(h_t, {c_s : s in S_t})           (Eq. 2, Fig. 1)
+ * The 128-d FP8 indexer key cache and the 512-d latent cache are the two
+ * per-token caches of "DeepSeek-V3.2开源技术报告" (nsmao.com, DSA principle).
+ *
+ * Conventions shared by every entry point
+ *  - All tensor arguments are device pointers to caller-owned memory,
+ *    row-major and dense, 16-byte aligned. The library allocates no memory.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream). Host-side argument checks return an error status
+ *    synchronously and launch nothing. Conditions only the device can see
+ *    (a sequence shorter than its query rows, a block-table entry outside the
+ *    cache, a bounded wait that ran out) set a device error word, read and
+ *    cleared by dsa_get_device_error(); the affected outputs are unspecified.
+ *  - The kernels are compiled for fixed dimensions: H^I = 64, d_I = 128,
+ *    H = 128 query heads, D = 576, D_v = 512, 1 <= k <= 2048, page size a
+ *    multiple of 64. Anything else returns DSA_ERR_UNSUPPORTED_SHAPE; there is
+ *    no fallback path.
+ *  - Query geometry: query row t belongs to sequence b = t / q_per_seq and sits
+ *    at position pos(t) = seqlen[b] - q_per_seq + (t % q_per_seq): the rows of a
+ *    sequence are its last q_per_seq tokens (decode: 1 or 2; prefill: all L).
+ *    Row t sees keys s in [0, pos(t)].
+ *  - Thread safety: calls may be issued from several host threads; calls
+ *    that overlap on the GPU share only the device error word.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+/* Same object as cudaStream_t; declared here so callers need no CUDA header. */
+typedef struct CUstream_st* dsa_stream_t;
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,       /* null pointer, bad size or alignment          */
+  DSA_ERR_UNSUPPORTED_SHAPE = 2, /* dims other than the compiled ones             */
+  DSA_ERR_CUDA = 3,              /* a CUDA runtime call failed                    */
+  DSA_ERR_DEVICE_TIMEOUT = 4,    /* a bounded device-side wait ran out            */
+  DSA_ERR_BOUNDS = 5,            /* device saw an index / page / length out of range */
+  DSA_ERR_WORKSPACE = 6          /* workspace missing or smaller than required    */
+} dsa_status_t;
+
+typedef enum { DSA_KV_CONTIGUOUS = 0, DSA_KV_PAGED = 1 } dsa_kv_layout_t;
+
+/* Geometry of the two per-token caches (indexer keys and MLA latents share it).
+ *  contiguous: token s of sequence b is row b * max_ctx + s of each cache array.
+ *  paged:      token s of sequence b is row (block_table[b][s / page_size]) *
+ *              page_size + s % page_size of each cache array. */
+typedef struct {
+  int32_t layout;              /* dsa_kv_layout_t                                       */
+  int32_t batch;               /* B sequences                                           */
+  int32_t max_ctx;             /* contiguous: token slots per sequence; paged: upper
+                                  bound on every seqlen (<= max_pages * page_size)      */
+  int32_t page_size;           /* paged only: tokens per page, a multiple of 64         */
+  int32_t num_pages;           /* paged only: physical pages in the cache arrays        */
+  int32_t max_pages;           /* paged only: columns of block_table                    */
+  const int32_t* block_table;  /* paged only: device int32 [batch][max_pages]           */
+  const int32_t* seqlens;      /* device int32 [batch]: tokens visible per sequence,
+                                  including its query rows; NULL = max_ctx for all      */
+} dsa_kv_desc_t;
+
+typedef struct {
+  int32_t num_q;               /* T = batch * q_per_seq                                 */
+  int32_t q_per_seq;           /* query rows per sequence (>= 1)                        */
+} dsa_q_desc_t;
+
+/* Lightning-indexer scores (Eq. 1 of the report, FP8 as its §1 allows).
+ *  q_idx   bf16 [T][64][128]  indexer queries; each (t, j) row is quantized on
+ *                             the fly to E4M3 with scale s_q = max(amax, 2^-120)/448
+ *  w       fp32 [T][64]       head weights w_{t,j}
+ *  k_idx   uint8 E4M3 codes, [B][max_ctx][128] or paged [num_pages][page_size][128]
+ *  k_scale fp32, [B][max_ctx] or paged [num_pages][page_size]: per-token key scale
+ *  scores  fp32 [T][ld] out:  scores[t][s] = s_k[s] * sum_j w_{t,j} s_q[t,j] *
+ *                             ReLU(q_hat_{t,j} . k_hat_s) for s <= pos(t), -inf for
+ *                             pos(t) < s < the end of the 128-key tile holding pos(t);
+ *                             later columns are not written.
+ *  ld      row stride of scores in elements, >= max_ctx rounded up to 128 and a
+ *          multiple of 4. */
+DSA_API dsa_status_t dsa_indexer_scores(const void* q_idx, const float* w, const void* k_idx,
+                                const float* k_scale, const dsa_kv_desc_t* kv,
+                                const dsa_q_desc_t* q, float* scores, int64_t ld,
+                                dsa_stream_t stream);
+
+/* Fine-grained token selection (report §1 and §2.1: S_t = Top-k(I_{t,:})).
+ *  scores fp32 [T][ld]: row t is read on [0, pos(t)] only.
+ *  idx    int32 [T][k] out: the k highest-scoring positions of row t in
+ *         ascending order; equal scores keep the lower position (-0.0 == +0.0);
+ *         when pos(t) + 1 <= k all visible positions are selected and the rest
+ *         of the row is -1. NaN scores are unsupported. */
+DSA_API dsa_status_t dsa_topk(const float* scores, int64_t ld, const dsa_kv_desc_t* kv,
+                      const dsa_q_desc_t* q, int32_t k, int32_t* idx, dsa_stream_t stream);
+
+/* Sparse MLA forward in MQA mode (report §1 Eq. 2, Fig. 1).
+ *  q     bf16 [T][128][576] absorbed queries
+ *  kv    bf16 latent cache, [B][max_ctx][576] or paged [num_pages][page_size][576]
+ *  idx   int32 [T][k]: logical token positions; entries outside [0, pos(t)]
+ *        (e.g. the -1 padding) are skipped; duplicates count as often as listed
+ *  scale softmax scale applied to q . c_s
+ *  out   bf16 [T][128][512] out: o_{t,h} = sum_s softmax_s(scale q_{t,h} . c_s) c_s[0:512]
+ *  lse   fp32 [T][128] out: ln sum_s exp(scale q_{t,h} . c_s); a row with no
+ *        valid entry gets o = 0 and lse = -inf. */
+DSA_API dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv_cache, const dsa_kv_desc_t* kv,
+                                const dsa_q_desc_t* qd, const int32_t* idx, int32_t k,
+                                float scale, void* out, float* lse, dsa_stream_t stream);
+
+/* Bytes of device workspace dsa_forward needs for this geometry (0 on a
+ * geometry the library rejects). */
+DSA_API size_t dsa_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k);
+
+/* The whole forward: indexer scores -> top-k -> sparse MLA, on `stream`.
+ * Arguments as in the three calls above. `workspace` (>= dsa_workspace_size
+ * bytes, 256-byte aligned) holds the score rows, processed in chunks of query
+ * rows when the full [T][max_ctx] matrix would not fit its bound, and the
+ * selected indices. idx_out (int32 [T][k]) receives the selection when not NULL. */
+DSA_API dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
+                         const float* k_scale, const void* q, const void* kv_cache,
+                         const dsa_kv_desc_t* kv, const dsa_q_desc_t* qd, int32_t k,
+                         float scale, void* workspace, size_t workspace_bytes,
+                         int32_t* idx_out, void* out, float* lse, dsa_stream_t stream);
+
+/* Synchronizes `stream`, then returns and clears the device error word
+ * (DSA_OK when no kernel reported a problem since the last call). */
+DSA_API dsa_status_t dsa_get_device_error(dsa_stream_t stream);
+
+/* Upper bound, in nanoseconds, on every bounded device-side wait (default
+ * 2e9). Returns the previous value. A value of 0 restores the default. */
+DSA_API uint64_t dsa_set_wait_timeout_ns(uint64_t ns);
+
+/* Launches one kernel whose bounded wait can never be satisfied, so that the
+ * timeout path is exercised without a fault: returns DSA_ERR_DEVICE_TIMEOUT
+ * (after about the configured timeout) when the path works. */
+DSA_API dsa_status_t dsa_selftest_wait_timeout(dsa_stream_t stream);
+
+/* Static description of a status code. */
+DSA_API const char* dsa_status_string(dsa_status_t status);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* DSA_H_ */

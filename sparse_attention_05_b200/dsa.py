@@ -1,0 +1,229 @@
+"""Thin Python binding of the C ABI in include/dsa.h (libdsa.so).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels. Tensors are PyTorch CUDA tensors (device memory and streams come from
+PyTorch); each call is enqueued on the current PyTorch stream unless a stream
+is given. There is no CPU or PyTorch fallback: a missing library raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa.so")
+
+DSA_KV_CONTIGUOUS = 0
+DSA_KV_PAGED = 1
+
+H_IDX, D_IDX, HEADS, D_QK, D_V, MAX_K = 64, 128, 128, 576, 512, 2048
+
+STATUS = {
+    0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED_SHAPE", 3: "DSA_ERR_CUDA",
+    4: "DSA_ERR_DEVICE_TIMEOUT", 5: "DSA_ERR_BOUNDS", 6: "DSA_ERR_WORKSPACE",
+}
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class KvDescC(ctypes.Structure):
+    _fields_ = [
+        ("layout", ctypes.c_int32), ("batch", ctypes.c_int32), ("max_ctx", ctypes.c_int32),
+        ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+        ("max_pages", ctypes.c_int32), ("block_table", ctypes.c_void_p),
+        ("seqlens", ctypes.c_void_p),
+    ]
+
+
+class QDescC(ctypes.Structure):
+    _fields_ = [("num_q", ctypes.c_int32), ("q_per_seq", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_lib = None
+
+# name -> (restype, argtypes): mirrors include/dsa.h
+SIGNATURES = {
+    "dsa_indexer_scores": (ctypes.c_int, [_P, _P, _P, _P, ctypes.POINTER(KvDescC),
+                                          ctypes.POINTER(QDescC), _P, ctypes.c_int64, _P]),
+    "dsa_topk": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.POINTER(KvDescC),
+                                ctypes.POINTER(QDescC), ctypes.c_int32, _P, _P]),
+    "dsa_sparse_mla_fwd": (ctypes.c_int, [_P, _P, ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
+                                          _P, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
+    "dsa_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
+                                             ctypes.c_int32]),
+    "dsa_forward": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.POINTER(KvDescC),
+                                   ctypes.POINTER(QDescC), ctypes.c_int32, ctypes.c_float, _P,
+                                   ctypes.c_size_t, _P, _P, _P, _P]),
+    "dsa_get_device_error": (ctypes.c_int, [_P]),
+    "dsa_set_wait_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
+    "dsa_selftest_wait_timeout": (ctypes.c_int, [_P]),
+    "dsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdsa.so (built in-tree by ``sparse_attention_05_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libdsa.so not built ({LIB_PATH}); run "
+                               "python -m sparse_attention_05_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise DSAError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the DSA library must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the DSA library must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+@dataclasses.dataclass
+class KvLayout:
+    """Geometry of the per-token caches (dsa_kv_desc_t)."""
+    batch: int
+    max_ctx: int
+    seqlens: Optional[torch.Tensor] = None         # int32 [batch] on the device
+    block_table: Optional[torch.Tensor] = None     # int32 [batch, max_pages] (paged)
+    page_size: int = 64
+    num_pages: int = 0
+
+    @property
+    def paged(self) -> bool:
+        return self.block_table is not None
+
+    def c(self) -> KvDescC:
+        d = KvDescC()
+        d.layout = DSA_KV_PAGED if self.paged else DSA_KV_CONTIGUOUS
+        d.batch, d.max_ctx = self.batch, self.max_ctx
+        d.page_size = self.page_size if self.paged else 0
+        d.num_pages = self.num_pages if self.paged else 0
+        d.max_pages = self.block_table.shape[1] if self.paged else 0
+        d.block_table = _ptr(self.block_table).value if self.paged else None
+        d.seqlens = _ptr(self.seqlens).value if self.seqlens is not None else None
+        return d
+
+    @staticmethod
+    def of(problem) -> "KvLayout":
+        """Geometry of a synth.Problem whose tensors live on the GPU."""
+        return KvLayout(batch=problem.batch, max_ctx=problem.max_ctx, seqlens=problem.seqlens,
+                        block_table=problem.block_table if problem.paged else None,
+                        page_size=problem.page_size,
+                        num_pages=problem.k_idx.shape[0] if problem.paged else 0)
+
+
+def _qdesc(num_q: int, q_per_seq: int) -> QDescC:
+    return QDescC(num_q, q_per_seq)
+
+
+def round_up(x: int, m: int) -> int:
+    return (x + m - 1) // m * m
+
+
+def dsa_indexer_scores(q_idx, w, k_idx, k_scale, kv: KvLayout, q_per_seq: int,
+                       scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    T = q_idx.shape[0]
+    if scores is None:
+        scores = torch.empty(T, round_up(kv.max_ctx, 128), dtype=torch.float32,
+                             device=q_idx.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq)
+    _check(lib().dsa_indexer_scores(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale),
+                                    ctypes.byref(kvd), ctypes.byref(qd), _ptr(scores),
+                                    scores.shape[1], _stream(stream)), "dsa_indexer_scores")
+    return scores
+
+
+def dsa_topk(scores, kv: KvLayout, q_per_seq: int, k: int,
+             idx: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    T = scores.shape[0]
+    if idx is None:
+        idx = torch.empty(T, k, dtype=torch.int32, device=scores.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq)
+    _check(lib().dsa_topk(_ptr(scores), scores.shape[1], ctypes.byref(kvd), ctypes.byref(qd), k,
+                          _ptr(idx), _stream(stream)), "dsa_topk")
+    return idx
+
+
+def dsa_sparse_mla_fwd(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale: float,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    T = q.shape[0]
+    if out is None:
+        out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq)
+    _check(lib().dsa_sparse_mla_fwd(_ptr(q), _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd),
+                                    _ptr(idx), idx.shape[1], float(scale), _ptr(out), _ptr(lse),
+                                    _stream(stream)), "dsa_sparse_mla_fwd")
+    return out, lse
+
+
+def dsa_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int) -> int:
+    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq)
+    return int(lib().dsa_workspace_size(ctypes.byref(kvd), ctypes.byref(qd), k))
+
+
+def dsa_forward(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_per_seq: int, k: int,
+                scale: float, workspace: Optional[torch.Tensor] = None,
+                idx_out: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                lse: Optional[torch.Tensor] = None, stream=None):
+    T = q.shape[0]
+    if workspace is None:
+        nbytes = dsa_workspace_size(kv, T, q_per_seq, k)
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq)
+    _check(lib().dsa_forward(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q),
+                             _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k, float(scale),
+                             _ptr(workspace), workspace.numel(), _ptr(idx_out), _ptr(out),
+                             _ptr(lse), _stream(stream)), "dsa_forward")
+    return out, lse, idx_out
+
+
+def dsa_get_device_error(stream=None) -> int:
+    return int(lib().dsa_get_device_error(_stream(stream)))
+
+
+def dsa_set_wait_timeout_ns(ns: int) -> int:
+    return int(lib().dsa_set_wait_timeout_ns(ns))
+
+
+def dsa_selftest_wait_timeout(stream=None) -> int:
+    return int(lib().dsa_selftest_wait_timeout(_stream(stream)))
+
+
+def dsa_status_string(status: int) -> str:
+    return lib().dsa_status_string(status).decode()
