@@ -1,0 +1,335 @@
+// indexer.cuh -- lightning indexer scores on the sm_100a tensor cores.
+//
+// DeepSeek-V3.2-Exp technical report (zh translation), §1 "Architecture", Eq. 1:
+//   I_{t,s} = sum_j w_{t,j} * ReLU(q^I_{t,j} . k^I_s),  keys s <= pos(t),
+// implemented in FP8 as that section allows: keys arrive as E4M3 codes with one
+// fp32 scale s_k per token; each (token, head) query row is quantized here to
+// E4M3 with s_q = max(amax, 2^-120) / 448, so that
+//   I_{t,s} = s_k[s] * sum_j (w_{t,j} s_q[t,j]) * ReLU(q_hat_{t,j} . k_hat_s).
+//
+// One persistent CTA per SM walks work units (sequence, group of G <= 4 query
+// rows, chunk of 128-key tiles). Per key tile the tensor core computes
+//   D[key][(row, head)] = K_tile (128 x 128 e4m3) . Q_group^T (64G x 128 e4m3)
+// into TMEM (M = 128 keys in lanes, N = 64G columns). The epilogue applies the
+// ReLU, the w*s_q-weighted head sum, the key scale and the causal mask straight
+// from TMEM, so the H^I x L x L intermediate never reaches memory; one fp32
+// score per (row, key) is stored.
+//
+// Warp roles (256 threads):
+//   warp 0      TMA producer: key tiles (2 boxes of 64 rows x 128 B, 128-B swizzle)
+//   warp 1      TMEM allocation + single-thread tcgen05.mma issue
+//   warps 2-3   query quantizers: bf16 -> E4M3 rows in the canonical swizzled
+//               K-major layout, w*s_q per row (double-buffered per unit)
+//   warps 4-7   epilogue, thread = key (TMEM lane), 2 accumulator buffers
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace dsa {
+
+constexpr int kIdxHeads = 64;
+constexpr int kIdxDim = 128;
+constexpr int kIdxTile = 128;                      // keys per tile (MMA M)
+constexpr int kIdxStages = 8;
+constexpr int kIdxThreads = 256;
+constexpr int kIdxStageBytes = kIdxTile * kIdxDim;  // 16 KB of e4m3
+constexpr int kIdxQBufBytes = 4 * kIdxHeads * kIdxDim;  // G <= 4 rows x 64 heads x 128 B
+constexpr int kIdxSmemBytes =
+    1024 /*align slack*/ + kIdxStages * kIdxStageBytes + 2 * kIdxQBufBytes +
+    2 * 4 * kIdxHeads * 4 /*wq*/ + 256 /*barriers etc*/;
+
+struct IndexerParams {
+  const __nv_bfloat16* q_idx;  // [T][64][128]
+  const float* w;              // [T][64]
+  const float* k_scale;        // [cache_rows]
+  const int32_t* block_table;  // [batch][max_pages] when paged
+  const int32_t* seqlens;      // [batch] or nullptr
+  float* scores;               // [batch * row_count][ld]
+  int64_t ld;
+  int32_t batch, max_ctx, q_per_seq;
+  int32_t paged, page_size, max_pages, num_pages;
+  int32_t row_begin, row_count;  // rows [row_begin, row_begin + row_count) of each sequence
+  int32_t G;                     // query rows per MMA (N = 64 G)
+  int32_t groups_per_seq;        // ceil(row_count / G)
+  int32_t chunk_tiles;           // key tiles per unit
+  int32_t chunks_per_group;
+  int64_t num_units;
+  uint64_t timeout_ns;
+};
+
+// Everything a role needs to know about one work unit; all roles derive it
+// identically from the unit index and the (read-only) sequence lengths.
+struct IdxUnit {
+  int b, i0, nrows, seqlen, kt0, kt1;  // key tiles [kt0, kt1)
+};
+
+__device__ __forceinline__ bool idx_unit(const IndexerParams& p, int64_t u, IdxUnit& U) {
+  const int64_t per_seq = (int64_t)p.groups_per_seq * p.chunks_per_group;
+  U.b = (int)(u / per_seq);
+  const int64_t rem = u - (int64_t)U.b * per_seq;
+  const int g = (int)(rem / p.chunks_per_group);
+  const int c = (int)(rem - (int64_t)g * p.chunks_per_group);
+  U.seqlen = p.seqlens ? __ldg(p.seqlens + U.b) : p.max_ctx;
+  if (U.seqlen < p.q_per_seq || U.seqlen > p.max_ctx) return false;  // reported by the epilogue
+  U.i0 = p.row_begin + g * p.G;
+  U.nrows = min(p.G, p.row_begin + p.row_count - U.i0);
+  const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
+  const int ntiles = pos_max / kIdxTile + 1;
+  U.kt0 = c * p.chunk_tiles;
+  U.kt1 = min(ntiles, U.kt0 + p.chunk_tiles);
+  return U.kt0 < U.kt1;
+}
+
+// Cache row of logical token s of sequence b (s must be < seqlen for paged).
+__device__ __forceinline__ int64_t idx_cache_row(const IndexerParams& p, int b, int s, bool& ok) {
+  ok = true;
+  if (!p.paged) return (int64_t)b * p.max_ctx + s;
+  const int page = __ldg(p.block_table + (int64_t)b * p.max_pages + s / p.page_size);
+  if (page < 0 || page >= p.num_pages) {
+    ok = false;
+    return 0;
+  }
+  return (int64_t)page * p.page_size + s % p.page_size;
+}
+
+__global__ void __launch_bounds__(kIdxThreads, 1)
+    indexer_kernel(const __grid_constant__ IndexerParams p,
+                   const __grid_constant__ CUtensorMap tm_keys) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint8_t* qbuf = stages + kIdxStages * kIdxStageBytes;
+  float* wq = reinterpret_cast<float*>(qbuf + 2 * kIdxQBufBytes);  // [2][256]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wq + 2 * 4 * kIdxHeads);
+  uint64_t* kfull = bars;
+  uint64_t* kempty = bars + kIdxStages;
+  uint64_t* tfull = bars + 2 * kIdxStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* qfull = tempty + 2;
+  uint64_t* qempty = qfull + 2;
+  uint64_t* mdone = qempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int N = kIdxHeads * p.G;
+  const uint32_t tmem_cols = N * 2 <= 128 ? 128 : (N * 2 <= 256 ? 256 : 512);
+
+  if (tid == 0) {
+    for (int s = 0; s < kIdxStages; ++s) {
+      mbar_init(smem_u32(&kfull[s]), 1);
+      mbar_init(smem_u32(&kempty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 128);
+      mbar_init(smem_u32(&qfull[i]), 64);
+      mbar_init(smem_u32(&qempty[i]), 1 + 128);
+    }
+    mbar_init(smem_u32(mdone), 1);
+    *abort_flag = 0;
+    fence_mbarrier_init_cluster();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint64_t TO = p.timeout_ns;
+  int drain_dummy = 0;
+  volatile int* no_abort = &drain_dummy;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_keys);
+      uint32_t it = 0;
+      for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+        IdxUnit U;
+        if (!idx_unit(p, u, U)) continue;
+        const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
+        for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
+          const int st = it % kIdxStages;
+          if (!mbar_wait(smem_u32(&kempty[st]), ((it / kIdxStages) & 1) ^ 1, TO, abort_flag))
+            break;
+          const uint32_t bar = smem_u32(&kfull[st]);
+          mbar_arrive_expect_tx(bar, kIdxStageBytes);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int s0 = kt * kIdxTile + h * 64;
+            int64_t row = 0;
+            if (s0 <= pos_max) {
+              bool ok;
+              row = idx_cache_row(p, U.b, s0, ok);
+              if (!ok) report_error(kErrBounds);
+            }
+            tma_load_2d(smem_u32(stages + st * kIdxStageBytes + h * 8192), &tm_keys, bar, 0,
+                        (int)row);
+          }
+        }
+      }
+      // Drain: the last stages' loads must land before the CTA may exit.
+      for (uint32_t j = it > kIdxStages ? it - kIdxStages : 0; j < it; ++j)
+        mbar_wait(smem_u32(&kfull[j % kIdxStages]), (j / kIdxStages) & 1, TO, no_abort);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = instr_desc(0 /*e4m3*/, 0, 0, 128, N);
+      uint32_t it = 0, un = 0;
+      for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+        IdxUnit U;
+        if (!idx_unit(p, u, U)) continue;
+        const int qb = un & 1;
+        if (!mbar_wait(smem_u32(&qfull[qb]), (un >> 1) & 1, TO, abort_flag)) break;
+        const uint32_t qaddr = smem_u32(qbuf + qb * kIdxQBufBytes);
+        bool ok = true;
+        for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
+          const int st = it % kIdxStages, ab = it & 1;
+          if (!mbar_wait(smem_u32(&kfull[st]), (it / kIdxStages) & 1, TO, abort_flag) ||
+              !mbar_wait(smem_u32(&tempty[ab]), ((it >> 1) & 1) ^ 1, TO, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kaddr = smem_u32(stages + st * kIdxStageBytes);
+          const uint32_t dcol = tmem_base + ab * N;
+#pragma unroll
+          for (int kk = 0; kk < kIdxDim / 32; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(kaddr + kk * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(qaddr + kk * 32, 16, 1024);
+            mma_fp8_ss(dcol, adesc, bdesc, idesc, kk > 0);
+          }
+          mma_commit(smem_u32(&kempty[st]));
+          mma_commit(smem_u32(&tfull[ab]));
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&qempty[qb]));
+        ++un;
+      }
+      // Every MMA issued above must finish before TMEM may be released.
+      mma_commit(smem_u32(mdone));
+      mbar_wait(smem_u32(mdone), 0, TO, no_abort);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ query quantizers
+    const int qw = warp - 2;  // 0..1
+    uint32_t un = 0;
+    for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+      IdxUnit U;
+      if (!idx_unit(p, u, U)) continue;
+      const int qb = un & 1;
+      if (!warp_wait(smem_u32(&qempty[qb]), ((un >> 1) & 1) ^ 1, TO, abort_flag)) break;
+      uint8_t* qdst = qbuf + qb * kIdxQBufBytes;
+      float* wdst = wq + qb * 4 * kIdxHeads;
+      for (int r = qw; r < N; r += 2) {
+        const int gi = r / kIdxHeads, j = r % kIdxHeads;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        float wj = 0.f;
+        if (gi < U.nrows) {
+          const int64_t t = (int64_t)U.b * p.q_per_seq + U.i0 + gi;
+          const uint2 raw = __ldg(reinterpret_cast<const uint2*>(
+              p.q_idx + (t * kIdxHeads + j) * kIdxDim + lane * 4));
+          x[0] = __uint_as_float(raw.x << 16);
+          x[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+          x[2] = __uint_as_float(raw.y << 16);
+          x[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+          wj = __ldg(p.w + t * kIdxHeads + j);
+        }
+        float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float sq = __fdiv_rn(fmaxf(amax, 0x1p-120f), 448.0f);
+        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[0], sq), __fdiv_rn(x[1], sq));
+        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[2], sq), __fdiv_rn(x[3], sq));
+        *reinterpret_cast<uint32_t*>(qdst + sw128_offset(r, lane >> 2) + (lane & 3) * 4) =
+            lo | (hi << 16);
+        if (lane == 0) wdst[r] = wj * sq;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&qfull[qb]));
+      ++un;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = tid - 128;           // key within the tile == TMEM lane
+    const int quad = warp - 4;         // TMEM lane quadrant of this warp
+    uint32_t it = 0, un = 0;
+    for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+      IdxUnit U;
+      if (!idx_unit(p, u, U)) {
+        const int b = (int)(u / ((int64_t)p.groups_per_seq * p.chunks_per_group));
+        const int sl = p.seqlens ? __ldg(p.seqlens + b) : p.max_ctx;
+        if (e == 0 && (sl < p.q_per_seq || sl > p.max_ctx)) report_error(kErrBounds);
+        continue;
+      }
+      const int qb = un & 1;
+      if (!warp_wait(smem_u32(&qfull[qb]), (un >> 1) & 1, TO, abort_flag)) break;
+      const float* wrow = wq + qb * 4 * kIdxHeads;
+      const int pos0 = U.seqlen - p.q_per_seq + U.i0;  // position of the group's first row
+      const int pos_max = pos0 + U.nrows - 1;
+      bool ok = true;
+      for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
+        const int ab = it & 1;
+        const int s = kt * kIdxTile + e;
+        float ks = 0.f;
+        if (s <= pos_max) {
+          bool rok;
+          const int64_t row = idx_cache_row(p, U.b, s, rok);
+          if (rok) ks = __ldg(p.k_scale + row);
+        }
+        if (!warp_wait(smem_u32(&tfull[ab]), (it >> 1) & 1, TO, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int gi = 0; gi < U.nrows; ++gi) {
+          float acc = 0.f;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + ab * N + gi * kIdxHeads +
+                          half * 32,
+                      v);
+            tmem_wait_ld();
+            const float4* w4 = reinterpret_cast<const float4*>(wrow + gi * kIdxHeads + half * 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const float4 ww = w4[q4];
+              acc = fmaf(ww.x, fmaxf(v[4 * q4 + 0], 0.f), acc);
+              acc = fmaf(ww.y, fmaxf(v[4 * q4 + 1], 0.f), acc);
+              acc = fmaf(ww.z, fmaxf(v[4 * q4 + 2], 0.f), acc);
+              acc = fmaf(ww.w, fmaxf(v[4 * q4 + 3], 0.f), acc);
+            }
+          }
+          const float out = (s <= pos0 + gi) ? ks * acc : -INFINITY;
+          const int64_t orow = (int64_t)U.b * p.row_count + (U.i0 - p.row_begin) + gi;
+          p.scores[orow * p.ld + s] = out;
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&tempty[ab]));
+      }
+      if (!ok) break;
+      mbar_arrive(smem_u32(&qempty[qb]));
+      ++un;
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+}  // namespace dsa
