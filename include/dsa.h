@@ -129,10 +129,13 @@ DSA_API dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv_cache, con
 DSA_API size_t dsa_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k);
 
 /* The whole forward: indexer scores -> top-k -> sparse MLA, on `stream`.
- * Arguments as in the three calls above. `workspace` (>= dsa_workspace_size
- * bytes, 256-byte aligned) holds the score rows, processed in chunks of query
- * rows when the full [T][max_ctx] matrix would not fit its bound, and the
- * selected indices. idx_out (int32 [T][k]) receives the selection when not NULL. */
+ * Arguments as in the three calls above. `workspace` (256-byte aligned) holds
+ * the selected indices (unless idx_out is given) and one chunk of score rows;
+ * dsa_workspace_size() bytes let the score rows go in chunks of up to 2 GiB. A
+ * smaller workspace is accepted down to the indices plus one score row per
+ * sequence; the rows are then processed in smaller chunks. Too small a
+ * workspace returns DSA_ERR_WORKSPACE. idx_out (int32 [T][k]) receives the
+ * selection when not NULL. */
 DSA_API dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
                          const float* k_scale, const void* q, const void* kv_cache,
                          const dsa_kv_desc_t* kv, const dsa_q_desc_t* qd, int32_t k,

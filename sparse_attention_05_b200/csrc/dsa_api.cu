@@ -20,7 +20,7 @@ using namespace dsa;
 
 namespace {
 
-constexpr int kHIdx = 64, kDIdx = 128, kHeads = 128, kDqk = 576, kDv = 512, kMaxK = 2048;
+constexpr int kDIdx = 128, kHeads = 128, kDqk = 576, kMaxK = 2048;
 
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 
@@ -96,9 +96,257 @@ dsa_status_t launch_topk(const float* scores, int64_t ld, const Geometry& g, int
   return cuda_status(cudaGetLastError());
 }
 
+// ---- TMA tensor maps ---------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// 2-D row-major tensor [rows][cols] with 128-byte swizzled boxes of box_rows x box_cols.
+dsa_status_t make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                          int elem_bytes, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                          uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return DSA_ERR_CUDA;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ---- indexer launch -----------------------------------------------------------------
+dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx,
+                            const float* k_scale, const Geometry& g, float* scores, int64_t ld,
+                            int row_begin, int row_count, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(indexer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kIdxSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  CUtensorMap tm;
+  dsa_status_t st = make_tmap_2d(&tm, k_idx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kDIdx,
+                                 (uint64_t)g.cache_rows, kDIdx, 64);
+  if (st != DSA_OK) return st;
+  IndexerParams p{};
+  p.q_idx = reinterpret_cast<const __nv_bfloat16*>(q_idx);
+  p.w = w;
+  p.k_scale = k_scale;
+  p.block_table = g.block_table;
+  p.seqlens = g.seqlens;
+  p.scores = scores;
+  p.ld = ld;
+  p.batch = g.batch;
+  p.max_ctx = g.max_ctx;
+  p.q_per_seq = g.q_per_seq;
+  p.paged = g.layout == DSA_KV_PAGED;
+  p.page_size = g.page_size;
+  p.max_pages = g.max_pages;
+  p.num_pages = g.num_pages;
+  p.row_begin = row_begin;
+  p.row_count = row_count;
+  p.G = std::min(4, row_count);
+  p.groups_per_seq = (row_count + p.G - 1) / p.G;
+  const int tiles = (g.max_ctx + kIdxTile - 1) / kIdxTile;
+  p.chunk_tiles = p.groups_per_seq == 1 ? 8 : tiles;
+  p.chunks_per_group = (tiles + p.chunk_tiles - 1) / p.chunk_tiles;
+  p.num_units = (int64_t)g.batch * p.groups_per_seq * p.chunks_per_group;
+  p.timeout_ns = g_timeout_ns.load();
+  if (p.num_units == 0) return DSA_OK;
+  const int grid = (int)std::min<int64_t>(p.num_units, num_sms());
+  indexer_kernel<<<grid, kIdxThreads, kIdxSmemBytes, stream>>>(p, tm);
+  return cuda_status(cudaGetLastError());
+}
+
+// ---- sparse MLA launch --------------------------------------------------------------
+dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geometry& g,
+                               const int32_t* idx, int k, float scale, void* out, float* lse,
+                               cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(sparse_mla_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  CUtensorMap tm;
+  dsa_status_t st = make_tmap_2d(&tm, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDqk,
+                                 (uint64_t)g.num_q * kHeads, 64, 128);
+  if (st != DSA_OK) return st;
+  MlaParams p{};
+  p.kv = reinterpret_cast<const uint8_t*>(kv_cache);
+  p.idx = idx;
+  p.block_table = g.block_table;
+  p.seqlens = g.seqlens;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.k = k;
+  p.batch = g.batch;
+  p.max_ctx = g.max_ctx;
+  p.q_per_seq = g.q_per_seq;
+  p.paged = g.layout == DSA_KV_PAGED;
+  p.page_size = g.page_size;
+  p.max_pages = g.max_pages;
+  p.num_pages = g.num_pages;
+  p.cache_rows = g.cache_rows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(2 * (int64_t)g.num_q), 1, 1);
+  cfg.blockDim = dim3(kMlaThreads, 1, 1);
+  cfg.dynamicSmemBytes = kMlaSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, sparse_mla_kernel, p, tm));
+}
+
+// ---- dsa_forward workspace plan --------------------------------------------------------
+constexpr int64_t kScoreBudgetBytes = 2ll << 30;  // bound on one chunk of score rows
+
+struct ForwardPlan {
+  int64_t ld;           // score row stride
+  int chunk_rows;       // query rows per sequence per chunk
+  size_t idx_bytes;     // selected indices (0 when the caller provides idx_out)
+  size_t score_bytes;   // one chunk of score rows
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+ForwardPlan plan_forward(const Geometry& g, int k, bool need_idx) {
+  ForwardPlan f;
+  f.ld = (int64_t)(g.max_ctx + kIdxTile - 1) / kIdxTile * kIdxTile;
+  const int64_t row_bytes = f.ld * 4 * g.batch;  // one row index across all sequences
+  int64_t rows = std::max<int64_t>(1, kScoreBudgetBytes / row_bytes);
+  if (rows >= g.q_per_seq) {
+    rows = g.q_per_seq;
+  } else if (rows >= 4) {
+    rows &= ~int64_t(3);  // whole groups of 4 rows per indexer MMA
+  }
+  f.chunk_rows = (int)rows;
+  f.idx_bytes = need_idx ? align256((size_t)g.num_q * k * 4) : 0;
+  f.score_bytes = align256((size_t)f.chunk_rows * row_bytes);
+  return f;
+}
+
+// ---- wait-timeout self test ---------------------------------------------------------
+__global__ void wait_timeout_selftest_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the bounded wait must give up and report
+  mbar_wait(smem_u32(&bar), 0, timeout_ns, &abort_flag);
+}
+
 }  // namespace
 
 extern "C" {
+
+dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv_cache, const dsa_kv_desc_t* kv,
+                                const dsa_q_desc_t* qd, const int32_t* idx, int32_t k,
+                                float scale, void* out, float* lse, dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !kv_cache || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!(scale > 0.f) || !(scale < 1e30f)) return DSA_ERR_INVALID_ARG;
+  return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, (cudaStream_t)stream);
+}
+
+size_t dsa_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k) {
+  Geometry g;
+  if (check_geometry(kv, q, &g) != DSA_OK || k < 1 || k > kMaxK) return 0;
+  const ForwardPlan f = plan_forward(g, k, true);
+  return f.idx_bytes + f.score_bytes;
+}
+
+dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
+                         const float* k_scale, const void* q, const void* kv_cache,
+                         const dsa_kv_desc_t* kv, const dsa_q_desc_t* qd, int32_t k,
+                         float scale, void* workspace, size_t workspace_bytes,
+                         int32_t* idx_out, void* out, float* lse, dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (!q_idx || !w || !k_idx || !k_scale || !q || !kv_cache || !out || !lse)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(kv_cache) ||
+      !aligned16(out))
+    return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!(scale > 0.f) || !(scale < 1e30f)) return DSA_ERR_INVALID_ARG;
+  ForwardPlan f = plan_forward(g, k, idx_out == nullptr);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < f.idx_bytes)
+    return DSA_ERR_WORKSPACE;
+  // A smaller workspace than dsa_workspace_size() is accepted: the score rows
+  // are then processed in smaller chunks (down to one row per sequence).
+  if (workspace_bytes < f.idx_bytes + f.score_bytes) {
+    const int64_t row_bytes = f.ld * 4 * g.batch;
+    int64_t rows = (int64_t)(workspace_bytes - f.idx_bytes) / row_bytes;
+    if (rows < 1) return DSA_ERR_WORKSPACE;
+    if (rows >= 4) rows &= ~int64_t(3);
+    f.chunk_rows = (int)rows;
+  }
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws);
+  float* scores = reinterpret_cast<float*>(ws + f.idx_bytes);
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int r0 = 0; r0 < g.q_per_seq; r0 += f.chunk_rows) {
+    const int rc = std::min(f.chunk_rows, g.q_per_seq - r0);
+    st = launch_indexer(q_idx, w, k_idx, k_scale, g, scores, f.ld, r0, rc, s);
+    if (st != DSA_OK) return st;
+    st = launch_topk(scores, f.ld, g, r0, rc, k, idx, s);
+    if (st != DSA_OK) return st;
+  }
+  return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, s);
+}
+
+dsa_status_t dsa_selftest_wait_timeout(dsa_stream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(g_timeout_ns.load());
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  return dsa_get_device_error(stream);
+}
+
+dsa_status_t dsa_indexer_scores(const void* q_idx, const float* w, const void* k_idx,
+                                const float* k_scale, const dsa_kv_desc_t* kv,
+                                const dsa_q_desc_t* q, float* scores, int64_t ld,
+                                dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, q, &g);
+  if (st != DSA_OK) return st;
+  if (!q_idx || !w || !k_idx || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  if (ld < (int64_t)(g.max_ctx + kIdxTile - 1) / kIdxTile * kIdxTile || ld % 4 != 0)
+    return DSA_ERR_INVALID_ARG;
+  return launch_indexer(q_idx, w, k_idx, k_scale, g, scores, ld, 0, g.q_per_seq,
+                        (cudaStream_t)stream);
+}
+
 
 const char* dsa_status_string(dsa_status_t s) {
   switch (s) {
@@ -144,19 +392,3 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, const dsa_kv_desc_t* kv,
 
 }  // extern "C"
 
-// TEMPORARY stubs (replaced as the kernels land)
-extern "C" {
-dsa_status_t dsa_indexer_scores(const void*, const float*, const void*, const float*,
-                                const dsa_kv_desc_t*, const dsa_q_desc_t*, float*, int64_t,
-                                dsa_stream_t) { return DSA_ERR_UNSUPPORTED_SHAPE; }
-dsa_status_t dsa_sparse_mla_fwd(const void*, const void*, const dsa_kv_desc_t*,
-                                const dsa_q_desc_t*, const int32_t*, int32_t, float, void*,
-                                float*, dsa_stream_t) { return DSA_ERR_UNSUPPORTED_SHAPE; }
-size_t dsa_workspace_size(const dsa_kv_desc_t*, const dsa_q_desc_t*, int32_t) { return 0; }
-dsa_status_t dsa_forward(const void*, const float*, const void*, const float*, const void*,
-                         const void*, const dsa_kv_desc_t*, const dsa_q_desc_t*, int32_t, float,
-                         void*, size_t, int32_t*, void*, float*, dsa_stream_t) {
-  return DSA_ERR_UNSUPPORTED_SHAPE;
-}
-dsa_status_t dsa_selftest_wait_timeout(dsa_stream_t) { return DSA_ERR_UNSUPPORTED_SHAPE; }
-}

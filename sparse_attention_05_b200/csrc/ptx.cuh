@@ -41,6 +41,20 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier over `nthreads` threads that also ANDs a predicate across them,
+// so that a group of warps takes one decision together.
+__device__ __forceinline__ bool named_barrier_and(int id, int nthreads, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{ .reg .pred pi, po; setp.ne.u32 pi, %3, 0;\n\t"
+      "barrier.red.and.pred po, %1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po; }"
+      : "=r"(out)
+      : "r"(id), "r"(nthreads), "r"(pred ? 1u : 0u)
+      : "memory");
+  return out != 0;
+}
+
 // ------------------------------------------------------------------------------------
 // mbarrier
 // ------------------------------------------------------------------------------------
