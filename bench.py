@@ -1,0 +1,528 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 DSA forward hot path (lightning indexer -> top-k ->
+sparse MLA) on synthetic inputs, one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole path over the workload's query rows with all
+inputs resident in device memory. The timed region (K steps) is bracketed by a
+barrier and a device synchronize, timed with CUDA events on the launching
+stream, and reduced as the max over ranks. Every rank runs the full workload
+on its own seeded inputs (independent sequences: weak scaling, no data-path
+collective). Per-kernel durations come from CUDA events around each launch
+inside the timed region. ``--impl reference`` times the CPU oracle on host
+cores on a bounded sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_05_b200 import synth  # noqa: E402
+
+METRIC = "DSA fwd query tokens/s at 128K ctx (decode & prefill); % of HBM / tensor roofline"
+UNIT = "query tokens/s"
+K_SEL = 2048
+
+WORKLOADS = {
+    # 128K-context decode: varlen paged cache, 2 query tokens per sequence
+    "paged_decode_128k": dict(kind="paged", batch=128, q_per_seq=2, min_ctx=4096,
+                              max_ctx=131072, page_size=64, seed=4),
+    "decode_32k": dict(kind="decode", batch=64, ctx=32768, q_per_seq=1, seed=1),
+    "prefill_8k": dict(kind="prefill", L=8192, seed=2),
+    "prefill_128k": dict(kind="prefill", L=131072, seed=3, n_hot=64),
+}
+DEFAULT_WORKLOAD = "paged_decode_128k"
+
+SCORE_BUDGET = 2 << 30  # bytes of fp32 score rows per chunk (as the library's own plan)
+
+
+# ----------------------------------------------------------------------------------------
+# workload and algorithmic work
+# ----------------------------------------------------------------------------------------
+def make_problem(name: str, device, seed_offset: int = 0) -> synth.Problem:
+    w = dict(WORKLOADS[name])
+    kind = w.pop("kind")
+    w["seed"] = w["seed"] + 1000 * seed_offset
+    if kind == "paged":
+        return synth.paged_decode(device=device, **w)
+    if kind == "decode":
+        return synth.decode(device=device, latent_std=0.5, **w)
+    return synth.prefill(device=device, **w)
+
+
+def algorithmic_work(p: synth.Problem, k: int = K_SEL) -> dict:
+    """Bytes and FLOPs the method must move or compute per step, per kernel.
+
+    indexer: 132 B per visible key per sequence (128 B E4M3 + 4 B scale), the
+             query rows (bf16) and weights, one fp32 score per (row, visible key);
+             16384 FP8 FLOP per (row, visible key).
+    top-k:   one read of each visible score, k int32 written per row.
+    sparse MLA: Q (bf16), out (bf16), LSE, indices, 1152 B per selected latent
+             row per query row; 278528 BF16 FLOP per (row, selected key).
+    """
+    seqlens = p.seqlens.cpu().long()
+    pos = p.q_pos().long()
+    n_vis = pos + 1
+    n_sel = torch.clamp(n_vis, max=k)
+    T = p.num_q
+    keys = int(seqlens.sum())  # every sequence's keys are read once
+    idx_bytes = 132 * keys + T * (64 * 128 * 2 + 64 * 4) + 4 * int(n_vis.sum())
+    idx_flop = 16384 * int(n_vis.sum())
+    topk_bytes = 4 * int(n_vis.sum()) + 4 * T * k
+    mla_bytes = T * (128 * 576 * 2 + 128 * 512 * 2 + 128 * 4 + 4 * k) + 1152 * int(n_sel.sum())
+    mla_flop = 278528 * int(n_sel.sum())
+    return {
+        "indexer": {"bytes": idx_bytes, "flop": idx_flop, "flop_dtype": "fp8"},
+        "topk": {"bytes": topk_bytes, "flop": 0, "flop_dtype": None},
+        "sparse_mla": {"bytes": mla_bytes, "flop": mla_flop, "flop_dtype": "bf16"},
+    }
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        m = json.load(open(path))
+        return {"hbm_gbs": m["hbm_gbs"], "bf16_tflops": m["bf16_tflops"],
+                "bf16_tflops_sustained": m.get("bf16_tflops_sustained", m["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def roofline(kernel: str, work: dict, avg_s: float, peaks: dict, long_step: bool) -> dict:
+    """Roofline of one kernel from its algorithmic work and average launch time."""
+    w = work[kernel]
+    bf16 = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
+    tflops = {"bf16": bf16, "fp8": 2.0 * bf16}  # FP8 = BF16 measured x nominal 4.5/2.25
+    t_mem = w["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_cmp = w["flop"] / (tflops[w["flop_dtype"]] * 1e12) if w["flop"] else 0.0
+    if t_cmp > t_mem:
+        achieved = w["flop"] / avg_s / 1e12
+        peak = tflops[w["flop_dtype"]]
+        r = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+             "dtype": w["flop_dtype"]}
+    else:
+        achieved = w["bytes"] / avg_s / 1e9
+        peak = peaks["hbm_gbs"]
+        r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s"}
+    r["frac"] = achieved / peak
+    r["peak_source"] = peaks["source"] + ("" if r["unit"] == "GB/s" else
+                                          (" sustained" if long_step else " burst") +
+                                          (" x2 (fp8 from bf16)" if w["flop_dtype"] == "fp8" else ""))
+    return r
+
+
+def dram_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it matches the
+    kernel source that is built now (else null)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        d = json.load(open(path))
+        e = d.get(workload, {}).get(kernel)
+        if not e:
+            return None
+        from sparse_attention_05_b200.build import source_digest
+        if e.get("source_digest") != source_digest():
+            return None
+        return e["bytes_per_launch"]
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            # select this process's GPU by UUID: nvidia-smi ignores CUDA_VISIBLE_DEVICES
+            gpu = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 6 and parts[0].isdigit():
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[2 + i] == "Active"})
+        return {"sm_mhz": statistics.median(float(r[0]) for r in rows),
+                "sm_max_mhz": float(rows[0][1]), "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------------
+class Runner:
+    """Holds the device buffers of one workload and runs one step of the path
+    through the library's stage calls (the same launches dsa_forward makes)."""
+
+    def __init__(self, p: synth.Problem, k: int = K_SEL):
+        from sparse_attention_05_b200 import dsa
+        self.dsa = dsa
+        self.p = p
+        self.k = k
+        self.kv = dsa.KvLayout.of(p)
+        T, B = p.num_q, p.batch
+        self.ld = dsa.round_up(p.max_ctx, 128)
+        rows = max(1, SCORE_BUDGET // (self.ld * 4 * B))
+        if rows >= p.q_per_seq:
+            rows = p.q_per_seq
+        elif rows >= 4:
+            rows &= ~3
+        self.chunks = [(r0, min(rows, p.q_per_seq - r0)) for r0 in range(0, p.q_per_seq, rows)]
+        self.scores = torch.empty(B * rows, self.ld, dtype=torch.float32, device=p.q.device)
+        self.idx = torch.empty(T, k, dtype=torch.int32, device=p.q.device)
+        self.out = torch.empty(T, 128, 512, dtype=torch.bfloat16, device=p.q.device)
+        self.lse = torch.empty(T, 128, dtype=torch.float32, device=p.q.device)
+        self.launches_per_step = 2 * len(self.chunks) + 1
+
+    def step(self, ev=None):
+        d, p = self.dsa, self.p
+        for r0, rc in self.chunks:
+            if ev is not None:
+                ev["indexer"].append(_record())
+            d.dsa_indexer_scores(p.q_idx, p.w, p.k_idx, p.k_scale, self.kv, p.q_per_seq,
+                                 scores=self.scores[: p.batch * rc], rows=(r0, rc))
+            if ev is not None:
+                ev["indexer"].append(_record())
+                ev["topk"].append(_record())
+            d.dsa_topk(self.scores[: p.batch * rc], self.kv, p.q_per_seq, self.k, idx=self.idx,
+                       rows=(r0, rc))
+            if ev is not None:
+                ev["topk"].append(_record())
+        if ev is not None:
+            ev["sparse_mla"].append(_record())
+        d.dsa_sparse_mla_fwd(p.q, p.kv, self.kv, p.q_per_seq, self.idx, p.scale, out=self.out,
+                             lse=self.lse)
+        if ev is not None:
+            ev["sparse_mla"].append(_record())
+
+
+def _record():
+    e = torch.cuda.Event(enable_timing=True)
+    e.record()
+    return e
+
+
+def _pairs_ms(evs):
+    return [evs[i].elapsed_time(evs[i + 1]) for i in range(0, len(evs), 2)]
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """Slowest rank's time: the whole job is as fast as its slowest GPU."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, rows_per_rank: int, steps: int, max_secs: float) -> float:
+    """Whole-job query tokens/s: every rank processed rows_per_rank rows per step."""
+    return world * rows_per_rank * steps / max_secs
+
+
+def e2e_run(r: Runner, steps: int, warmup: int, world: int):
+    """Through the public call dsa_forward, with the step's query-side inputs
+    copied from pinned host memory and the result read back every step."""
+    d, p = r.dsa, r.p
+    host = {n: getattr(p, n).cpu().pin_memory() for n in ("q_idx", "w", "q", "seqlens")}
+    if p.paged:
+        host["block_table"] = p.block_table.cpu().pin_memory()
+    dev = {n: torch.empty_like(v, device="cuda") for n, v in host.items()}
+    out_h = torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory()
+    lse_h = torch.empty(r.lse.shape, dtype=r.lse.dtype).pin_memory()
+    ws = torch.empty(max(256, d.dsa_workspace_size(r.kv, p.num_q, p.q_per_seq, r.k)),
+                     dtype=torch.uint8, device="cuda")
+    kv = d.KvLayout(batch=p.batch, max_ctx=p.max_ctx, seqlens=dev["seqlens"],
+                    block_table=dev.get("block_table"), page_size=p.page_size,
+                    num_pages=r.kv.num_pages)
+
+    def one():
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        d.dsa_forward(dev["q_idx"], dev["w"], p.k_idx, p.k_scale, dev["q"], p.kv, kv,
+                      p.q_per_seq, r.k, p.scale, workspace=ws, out=r.out, lse=r.lse)
+        out_h.copy_(r.out, non_blocking=True)
+        lse_h.copy_(r.lse, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = _record()
+    for _ in range(steps):
+        one()
+    t1 = _record()
+    torch.cuda.synchronize()
+    barrier(world)
+    secs = max_over_ranks(t0.elapsed_time(t1) / 1e3, world)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    return {"value": job_throughput(world, p.num_q, steps, secs), "unit": UNIT,
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * secs / steps}
+
+
+# ----------------------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ----------------------------------------------------------------------------------------
+def oracle_sample_inputs(p: synth.Problem, rows):
+    """numpy inputs for the oracle restricted to the sequences of ``rows``,
+    each rebuilt contiguously on the host (pages resolved through the block
+    table), plus the rows' indices in that reduced problem."""
+    seqs = sorted({int(t) // p.q_per_seq for t in rows})
+    seqlens = p.seqlens.cpu().long()
+    ctx = int(max(seqlens[s] for s in seqs))
+    kc = np.zeros((len(seqs), ctx, 128), np.uint8)
+    ks = np.zeros((len(seqs), ctx), np.float32)
+    kvc = np.zeros((len(seqs), ctx, 576), np.float32)
+    for i, s in enumerate(seqs):
+        n = int(seqlens[s])
+        if p.paged:
+            pages = p.block_table[s, : (n + p.page_size - 1) // p.page_size].long()
+            kc[i, :n] = p.k_idx[pages].reshape(-1, 128)[:n].cpu().numpy()
+            ks[i, :n] = p.k_scale[pages].reshape(-1)[:n].cpu().numpy()
+            kvc[i, :n] = p.kv[pages].reshape(-1, 576)[:n].float().cpu().numpy()
+        else:
+            kc[i, :n] = p.k_idx[s, :n].cpu().numpy()
+            ks[i, :n] = p.k_scale[s, :n].cpu().numpy()
+            kvc[i, :n] = p.kv[s, :n].float().cpu().numpy()
+    trows = torch.as_tensor(list(rows))
+    q_seq = np.array([seqs.index(int(t) // p.q_per_seq) for t in rows])
+    q_pos = p.q_pos()[trows].numpy()
+    return dict(q_idx=p.q_idx[trows].float().cpu().numpy(), w=p.w[trows].cpu().numpy(),
+                k_idx=kc, k_scale=ks, q=p.q[trows].float().cpu().numpy(), kv=kvc,
+                q_seq=q_seq, q_pos=q_pos, ld=ctx)
+
+
+def oracle_step(inp, scale, k=K_SEL):
+    from oracle import dsa_forward as oracle_forward
+    return oracle_forward(inp["q_idx"], inp["w"], inp["k_idx"], inp["k_scale"], inp["q"],
+                          inp["kv"], inp["q_seq"], inp["q_pos"], k=k, scale=scale, d_v=512,
+                          ld=inp["ld"])
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(p: synth.Problem, name: str, budget_s: float = 12.0, seed: int = 0) -> dict:
+    rng = np.random.default_rng(seed)
+    rows_done, elapsed, seqs = 0, 0.0, []
+    while elapsed < budget_s and rows_done < p.num_q:
+        b = int(rng.integers(0, p.batch))
+        r0 = b * p.q_per_seq
+        rows = list(range(r0, r0 + min(p.q_per_seq, 2)))
+        inp = oracle_sample_inputs(p, rows)
+        t0 = time.perf_counter()
+        oracle_step(inp, p.scale)
+        elapsed += time.perf_counter() - t0
+        rows_done += len(rows)
+        seqs.append(b)
+    return {"value": rows_done / elapsed, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows_done} query rows of {name} (sequences {seqs[:8]}"
+                      f"{'...' if len(seqs) > 8 else ''}), full indexer+top-k+attention per row, "
+                      f"{elapsed:.1f} s of host time"}
+
+
+def reference_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    p = make_problem(args.workload, dev)
+    rng = np.random.default_rng(123)
+    per_step_rows = min(p.q_per_seq, 2)
+
+    def one():
+        b = int(rng.integers(0, p.batch))
+        rows = list(range(b * p.q_per_seq, b * p.q_per_seq + per_step_rows))
+        inp = oracle_sample_inputs(p, rows)
+        t0 = time.perf_counter()
+        oracle_step(inp, p.scale)
+        return time.perf_counter() - t0
+
+    for _ in range(args.warmup):
+        one()
+    secs = sum(one() for _ in range(args.steps))
+    value = args.steps * per_step_rows / secs
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, **WORKLOADS[args.workload],
+                       "sample_rows_per_step": per_step_rows},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"{per_step_rows} query rows of one random sequence per "
+                                       f"step, {args.steps} steps"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------------------
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--soak-s", type=float, default=1.0,
+                    help="untimed seconds of steps right before the timed region (clock samples)")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    world, rank, local = dist_setup(args.gpus)
+    p = make_problem(args.workload, "cuda", seed_offset=rank)
+    r = Runner(p)
+    work = algorithmic_work(p)
+    peaks = load_peaks()
+
+    for _ in range(args.warmup):
+        r.step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < args.soak_s:
+        r.step()
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = {"indexer": [], "topk": [], "sparse_mla": []}
+    start = _record()
+    for _ in range(args.steps):
+        r.step(ev)
+    stop = _record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    secs_local = start.elapsed_time(stop) / 1e3
+    secs = max_over_ranks(secs_local, world)
+
+    per_kernel = {kname: _pairs_ms(e) for kname, e in ev.items()}
+    launches = {kname: len(v) for kname, v in per_kernel.items()}
+    total_ms = {kname: sum(v) for kname, v in per_kernel.items()}
+    dominant = max(total_ms, key=total_ms.get)
+    long_step = secs / args.steps > 0.05
+    avg_s = total_ms[dominant] / 1e3 / args.steps  # one step's worth of that kernel
+    roof = roofline(dominant, work, avg_s, peaks, long_step)
+    roof["kernel"] = dominant
+    roof["launches_per_step"] = launches[dominant] // args.steps
+    roof["traffic"] = dram_traffic(dominant, args.workload)
+    stages = {}
+    for kname in per_kernel:
+        a = total_ms[kname] / 1e3 / args.steps
+        rf = roofline(kname, work, a, peaks, long_step)
+        stages[kname] = {"ms_per_step": 1e3 * a, "share": total_ms[kname] / sum(total_ms.values()),
+                         "bound": rf["bound"], "frac": rf["frac"],
+                         "achieved": rf["achieved"], "unit": rf["unit"]}
+
+    e2e = None if args.no_e2e else e2e_run(r, max(3, args.steps // 2), 3, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(p, args.workload)
+
+    if rank == 0:
+        cfg = {"workload": args.workload, **WORKLOADS[args.workload], "k": K_SEL,
+               "heads": 128, "d_qk": 576, "d_v": 512, "h_idx": 64, "d_idx": 128,
+               "query_rows_per_gpu": p.num_q,
+               "l2": "inputs larger than L2 (no flush)",
+               "parallelism": f"dp{world} (independent sequences per GPU)"}
+        line = {
+            "metric": METRIC, "value": job_throughput(world, p.num_q, args.steps, secs),
+            "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3+bf16", "data": "synthetic", "config": cfg,
+            "roofline": roof, "stages": stages, "clocks": clk,
+            "gpu_launches": sum(launches.values()),
+            "e2e": e2e, "cpu_baseline": cpu, "peaks": peaks,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

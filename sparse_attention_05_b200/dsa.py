@@ -45,7 +45,8 @@ class KvDescC(ctypes.Structure):
 
 
 class QDescC(ctypes.Structure):
-    _fields_ = [("num_q", ctypes.c_int32), ("q_per_seq", ctypes.c_int32)]
+    _fields_ = [("num_q", ctypes.c_int32), ("q_per_seq", ctypes.c_int32),
+                ("row_begin", ctypes.c_int32), ("row_count", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -141,21 +142,31 @@ class KvLayout:
                         num_pages=problem.k_idx.shape[0] if problem.paged else 0)
 
 
-def _qdesc(num_q: int, q_per_seq: int) -> QDescC:
-    return QDescC(num_q, q_per_seq)
+def _qdesc(num_q: int, q_per_seq: int, rows: Optional[Tuple[int, int]] = None) -> QDescC:
+    """rows = (row_begin, row_count) window within each sequence (None = all)."""
+    r0, rc = rows if rows is not None else (0, 0)
+    return QDescC(num_q, q_per_seq, r0, rc)
 
 
 def round_up(x: int, m: int) -> int:
     return (x + m - 1) // m * m
 
 
+def _window(kv: KvLayout, q_per_seq: int, rows) -> int:
+    """Rows per sequence covered by the window."""
+    r0, rc = rows if rows is not None else (0, 0)
+    return rc if rc else q_per_seq - r0
+
+
 def dsa_indexer_scores(q_idx, w, k_idx, k_scale, kv: KvLayout, q_per_seq: int,
-                       scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                       scores: Optional[torch.Tensor] = None, rows=None,
+                       stream=None) -> torch.Tensor:
+    """Scores [batch * window_rows, ld] (window rows stored compactly)."""
     T = q_idx.shape[0]
     if scores is None:
-        scores = torch.empty(T, round_up(kv.max_ctx, 128), dtype=torch.float32,
-                             device=q_idx.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq)
+        scores = torch.empty(kv.batch * _window(kv, q_per_seq, rows), round_up(kv.max_ctx, 128),
+                             dtype=torch.float32, device=q_idx.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
     _check(lib().dsa_indexer_scores(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale),
                                     ctypes.byref(kvd), ctypes.byref(qd), _ptr(scores),
                                     scores.shape[1], _stream(stream)), "dsa_indexer_scores")
@@ -163,11 +174,12 @@ def dsa_indexer_scores(q_idx, w, k_idx, k_scale, kv: KvLayout, q_per_seq: int,
 
 
 def dsa_topk(scores, kv: KvLayout, q_per_seq: int, k: int,
-             idx: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    T = scores.shape[0]
+             idx: Optional[torch.Tensor] = None, rows=None, stream=None) -> torch.Tensor:
+    """Selected positions [T, k] (rows outside the window are left untouched)."""
+    T = kv.batch * q_per_seq
     if idx is None:
         idx = torch.empty(T, k, dtype=torch.int32, device=scores.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
     _check(lib().dsa_topk(_ptr(scores), scores.shape[1], ctypes.byref(kvd), ctypes.byref(qd), k,
                           _ptr(idx), _stream(stream)), "dsa_topk")
     return idx
@@ -175,37 +187,37 @@ def dsa_topk(scores, kv: KvLayout, q_per_seq: int, k: int,
 
 def dsa_sparse_mla_fwd(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale: float,
                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                       stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                       rows=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     T = q.shape[0]
     if out is None:
         out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
     _check(lib().dsa_sparse_mla_fwd(_ptr(q), _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd),
                                     _ptr(idx), idx.shape[1], float(scale), _ptr(out), _ptr(lse),
                                     _stream(stream)), "dsa_sparse_mla_fwd")
     return out, lse
 
 
-def dsa_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int) -> int:
-    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq)
+def dsa_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None) -> int:
+    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows)
     return int(lib().dsa_workspace_size(ctypes.byref(kvd), ctypes.byref(qd), k))
 
 
 def dsa_forward(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_per_seq: int, k: int,
                 scale: float, workspace: Optional[torch.Tensor] = None,
                 idx_out: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                lse: Optional[torch.Tensor] = None, stream=None):
+                lse: Optional[torch.Tensor] = None, rows=None, stream=None):
     T = q.shape[0]
     if workspace is None:
-        nbytes = dsa_workspace_size(kv, T, q_per_seq, k)
+        nbytes = dsa_workspace_size(kv, T, q_per_seq, k, rows)
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
     _check(lib().dsa_forward(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q),
                              _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k, float(scale),
                              _ptr(workspace), workspace.numel(), _ptr(idx_out), _ptr(out),

@@ -1,0 +1,140 @@
+"""CPU checks of the C ABI (no GPU needed): the library builds and loads, exports
+every entry point include/dsa.h declares, the Python binding mirrors the header
+and its struct layouts, and the host-side argument checks return the documented
+status codes without launching anything."""
+
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"DSA_API\s+[\w\s\*]+?\b(dsa_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_05_b200.build import build
+    build()
+    from sparse_attention_05_b200 import dsa
+    return dsa.lib()
+
+
+def test_header_declares_the_four_path_calls():
+    names = _declared()
+    for n in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from sparse_attention_05_b200 import dsa
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(dsa_\w+)", out))
+    missing = set(_declared()) - exported
+    assert not missing, f"not exported: {missing}"
+
+
+def test_binding_mirrors_header():
+    from sparse_attention_05_b200 import dsa
+    assert sorted(dsa.SIGNATURES) == _declared()
+
+
+def test_struct_layouts_match_c():
+    from sparse_attention_05_b200 import dsa
+    src = r"""
+    #include <stdio.h>
+    #include <stddef.h>
+    #include "dsa.h"
+    int main(void) {
+      printf("%zu %zu %zu %zu %zu\n", sizeof(dsa_kv_desc_t), offsetof(dsa_kv_desc_t, block_table),
+             offsetof(dsa_kv_desc_t, seqlens), sizeof(dsa_q_desc_t), offsetof(dsa_q_desc_t, row_count));
+      return 0;
+    }
+    """
+    with tempfile.TemporaryDirectory() as d:
+        c, exe = os.path.join(d, "l.c"), os.path.join(d, "l")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
+        got = [int(x) for x in subprocess.run([exe], capture_output=True, text=True).stdout.split()]
+    want = [ctypes.sizeof(dsa.KvDescC), dsa.KvDescC.block_table.offset, dsa.KvDescC.seqlens.offset,
+            ctypes.sizeof(dsa.QDescC), dsa.QDescC.row_count.offset]
+    assert got == want
+
+
+def test_status_strings_and_timeout_setting(lib):
+    from sparse_attention_05_b200 import dsa
+    assert dsa.dsa_status_string(0) == "DSA_OK"
+    assert "TIMEOUT" in dsa.dsa_status_string(4)
+    old = dsa.dsa_set_wait_timeout_ns(123)
+    assert dsa.dsa_set_wait_timeout_ns(old) == 123
+
+
+def _kv(batch=2, max_ctx=512, layout=0, page=64, pages=0, max_pages=0, bt=None):
+    from sparse_attention_05_b200 import dsa
+    d = dsa.KvDescC()
+    d.layout, d.batch, d.max_ctx = layout, batch, max_ctx
+    d.page_size, d.num_pages, d.max_pages = page, pages, max_pages
+    d.block_table = bt
+    d.seqlens = None
+    return d
+
+
+def test_host_argument_checks_without_gpu(lib):
+    from sparse_attention_05_b200 import dsa
+    L = lib
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: the checks fail first
+    kv, q = _kv(), dsa.QDescC(2, 1, 0, 0)
+    by = ctypes.byref
+    # null output
+    assert L.dsa_topk(fake, 512, by(kv), by(q), 2048, None, None) == 1
+    # k out of range
+    assert L.dsa_topk(fake, 512, by(kv), by(q), 4096, fake, None) == 2
+    assert L.dsa_topk(fake, 512, by(kv), by(q), 0, fake, None) == 2
+    # T != batch * q_per_seq
+    bad_q = dsa.QDescC(3, 1, 0, 0)
+    assert L.dsa_topk(fake, 512, by(kv), by(bad_q), 2048, fake, None) == 1
+    # row window outside the sequence
+    assert L.dsa_topk(fake, 512, by(kv), by(dsa.QDescC(2, 1, 1, 0)), 2048, fake, None) == 1
+    # ld below max_ctx rounded to 128
+    assert L.dsa_indexer_scores(fake, fake, fake, fake, by(kv), by(q), fake, 500, None) == 1
+    # misaligned pointer
+    assert L.dsa_indexer_scores(ctypes.c_void_p(0x1001), fake, fake, fake, by(kv), by(q), fake,
+                                512, None) == 1
+    # paged: page size not a multiple of 64, missing block table
+    pk = _kv(layout=1, page=48, pages=4, max_pages=16, bt=0x2000)
+    assert L.dsa_sparse_mla_fwd(fake, fake, by(pk), by(q), fake, 2048, 0.04, fake, fake, None) == 2
+    pk = _kv(layout=1, page=64, pages=4, max_pages=16, bt=None)
+    assert L.dsa_sparse_mla_fwd(fake, fake, by(pk), by(q), fake, 2048, 0.04, fake, fake, None) == 1
+    # scale must be positive and finite
+    assert L.dsa_sparse_mla_fwd(fake, fake, by(kv), by(q), fake, 2048, -1.0, fake, fake, None) == 1
+    # workspace too small / misaligned
+    ws_need = L.dsa_workspace_size(by(kv), by(q), 2048)
+    assert ws_need >= 2 * 2048 * 4
+    assert L.dsa_forward(fake, fake, fake, fake, fake, fake, by(kv), by(q), 2048, 0.04,
+                         ctypes.c_void_p(0x1000), 16, None, fake, fake, None) == 6
+    assert L.dsa_forward(fake, fake, fake, fake, fake, fake, by(kv), by(q), 2048, 0.04,
+                         ctypes.c_void_p(0x1010), ws_need, None, fake, fake, None) == 6
+
+
+def test_workspace_size_plan(lib):
+    from sparse_attention_05_b200 import dsa
+    by = ctypes.byref
+    # decode, 64 x 32768: indices + all score rows in one chunk
+    kv, q = _kv(batch=64, max_ctx=32768), dsa.QDescC(64, 1, 0, 0)
+    n = lib.dsa_workspace_size(by(kv), by(q), 2048)
+    assert n == 64 * 2048 * 4 + 64 * 32768 * 4
+    # prefill 131072: indices + one 2 GiB chunk of score rows
+    kv, q = _kv(batch=1, max_ctx=131072), dsa.QDescC(131072, 131072, 0, 0)
+    n = lib.dsa_workspace_size(by(kv), by(q), 2048)
+    assert n == 131072 * 2048 * 4 + 4096 * 131072 * 4
+    # invalid geometry -> 0
+    assert lib.dsa_workspace_size(by(kv), by(dsa.QDescC(5, 131072, 0, 0)), 2048) == 0
