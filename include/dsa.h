@@ -80,9 +80,17 @@ typedef struct {
                                   including its query rows; NULL = max_ctx for all      */
 } dsa_kv_desc_t;
 
+/* Query rows. Each call processes the window of rows i in [row_begin,
+ * row_begin + row_count) of every sequence (row_count = 0 means all rows from
+ * row_begin on); rows outside the window are neither read nor written. Score
+ * rows are stored compactly per window: window row i of sequence b is score
+ * row b * row_count + (i - row_begin). Indices, queries, outputs and LSE keep
+ * their global row t = b * q_per_seq + i. */
 typedef struct {
   int32_t num_q;               /* T = batch * q_per_seq                                 */
   int32_t q_per_seq;           /* query rows per sequence (>= 1)                        */
+  int32_t row_begin;           /* first row of the window (0 = from the first row)      */
+  int32_t row_count;           /* rows in the window (0 = through the last row)         */
 } dsa_q_desc_t;
 
 /* Lightning-indexer scores (Eq. 1 of the report, FP8 as its §1 allows).
@@ -91,7 +99,8 @@ typedef struct {
  *  w       fp32 [T][64]       head weights w_{t,j}
  *  k_idx   uint8 E4M3 codes, [B][max_ctx][128] or paged [num_pages][page_size][128]
  *  k_scale fp32, [B][max_ctx] or paged [num_pages][page_size]: per-token key scale
- *  scores  fp32 [T][ld] out:  scores[t][s] = s_k[s] * sum_j w_{t,j} s_q[t,j] *
+ *  scores  fp32 [batch * row_count][ld] out (see dsa_q_desc_t for the row order):
+ *                             scores[t][s] = s_k[s] * sum_j w_{t,j} s_q[t,j] *
  *                             ReLU(q_hat_{t,j} . k_hat_s) for s <= pos(t), -inf for
  *                             pos(t) < s < the end of the 128-key tile holding pos(t);
  *                             later columns are not written.
@@ -103,7 +112,8 @@ DSA_API dsa_status_t dsa_indexer_scores(const void* q_idx, const float* w, const
                                 dsa_stream_t stream);
 
 /* Fine-grained token selection (report §1 and §2.1: S_t = Top-k(I_{t,:})).
- *  scores fp32 [T][ld]: row t is read on [0, pos(t)] only.
+ *  scores fp32 [batch * row_count][ld] as dsa_indexer_scores writes it: the
+ *         row of query t is read on [0, pos(t)] only.
  *  idx    int32 [T][k] out: the k highest-scoring positions of row t in
  *         ascending order; equal scores keep the lower position (-0.0 == +0.0);
  *         when pos(t) + 1 <= k all visible positions are selected and the rest
@@ -141,6 +151,33 @@ DSA_API dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* 
                          const dsa_kv_desc_t* kv, const dsa_q_desc_t* qd, int32_t k,
                          float scale, void* workspace, size_t workspace_bytes,
                          int32_t* idx_out, void* out, float* lse, dsa_stream_t stream);
+
+/* dsa_forward without a workspace argument, for callers that cannot allocate
+ * device memory themselves: for example a plugin that its host framework hands
+ * only input and output buffers, or a runtime whose device memory all belongs
+ * to its own pool allocator, so that neither cudaMalloc nor a framework
+ * allocator may be called for scratch space. (The technical report has no
+ * counterpart of this call; it is an interface convenience.)
+ *  - The scratch space is a fixed 128 MiB device array inside this library;
+ *    every GPU that loads the library holds it until the process exits. The
+ *    call allocates nothing.
+ *  - It must hold the selected indices (T * k * 4 bytes, none when idx_out is
+ *    given) plus at least one score row per sequence (round_up(max_ctx, 128) * 4
+ *    * batch bytes); larger geometries return DSA_ERR_WORKSPACE before anything
+ *    is launched. Score rows are processed in chunks that fit.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture begins.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents (nothing in it needs to start at zero). Calls whose kernels
+ *    overlap on the GPU, e.g. on two streams at once, race on it: serialize them.
+ * Arguments and results are those of dsa_forward. */
+DSA_API dsa_status_t dsa_forward_noalloc(const void* q_idx, const float* w, const void* k_idx,
+                                         const float* k_scale, const void* q,
+                                         const void* kv_cache, const dsa_kv_desc_t* kv,
+                                         const dsa_q_desc_t* qd, int32_t k, float scale,
+                                         int32_t* idx_out, void* out, float* lse,
+                                         dsa_stream_t stream);
 
 /* Synchronizes `stream`, then returns and clears the device error word
  * (DSA_OK when no kernel reported a problem since the last call). */

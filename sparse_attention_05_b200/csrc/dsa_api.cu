@@ -31,6 +31,7 @@ dsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA
 // Validated geometry shared by every entry point.
 struct Geometry {
   int layout, batch, max_ctx, page_size, num_pages, max_pages, q_per_seq, num_q;
+  int row_begin, row_count;  // window of rows per sequence
   const int32_t* block_table;
   const int32_t* seqlens;
   int64_t cache_rows;  // rows of each per-token cache array
@@ -41,6 +42,11 @@ dsa_status_t check_geometry(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, Geom
   if (kv->batch < 1 || kv->max_ctx < 1 || q->q_per_seq < 1) return DSA_ERR_INVALID_ARG;
   if ((int64_t)kv->batch * q->q_per_seq != q->num_q) return DSA_ERR_INVALID_ARG;
   if (q->q_per_seq > kv->max_ctx) return DSA_ERR_INVALID_ARG;
+  if (q->row_begin < 0 || q->row_begin >= q->q_per_seq || q->row_count < 0 ||
+      q->row_count > q->q_per_seq - q->row_begin)
+    return DSA_ERR_INVALID_ARG;
+  g->row_begin = q->row_begin;
+  g->row_count = q->row_count ? q->row_count : q->q_per_seq - q->row_begin;
   g->layout = kv->layout;
   g->batch = kv->batch;
   g->max_ctx = kv->max_ctx;
@@ -202,10 +208,12 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
   p.max_pages = g.max_pages;
   p.num_pages = g.num_pages;
   p.cache_rows = g.cache_rows;
+  p.row_begin = g.row_begin;
+  p.row_count = g.row_count;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns.load();
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(2 * (int64_t)g.num_q), 1, 1);
+  cfg.gridDim = dim3((unsigned)(2 * (int64_t)g.batch * g.row_count), 1, 1);
   cfg.blockDim = dim3(kMlaThreads, 1, 1);
   cfg.dynamicSmemBytes = kMlaSmemBytes;
   cfg.stream = stream;
@@ -236,8 +244,8 @@ ForwardPlan plan_forward(const Geometry& g, int k, bool need_idx) {
   f.ld = (int64_t)(g.max_ctx + kIdxTile - 1) / kIdxTile * kIdxTile;
   const int64_t row_bytes = f.ld * 4 * g.batch;  // one row index across all sequences
   int64_t rows = std::max<int64_t>(1, kScoreBudgetBytes / row_bytes);
-  if (rows >= g.q_per_seq) {
-    rows = g.q_per_seq;
+  if (rows >= g.row_count) {
+    rows = g.row_count;
   } else if (rows >= 4) {
     rows &= ~int64_t(3);  // whole groups of 4 rows per indexer MMA
   }
@@ -245,6 +253,30 @@ ForwardPlan plan_forward(const Geometry& g, int k, bool need_idx) {
   f.idx_bytes = need_idx ? align256((size_t)g.num_q * k * 4) : 0;
   f.score_bytes = align256((size_t)f.chunk_rows * row_bytes);
   return f;
+}
+
+// ---- scratch for the allocation-free forward ------------------------------------------
+// A fixed device array that every device loading this library holds until exit.
+// Host code must not use the symbol's host-side address: the device address is
+// resolved with cudaGetSymbolAddress, once per device, with that device current.
+constexpr size_t kStaticScratchBytes = size_t(128) << 20;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+dsa_status_t static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return DSA_OK;
 }
 
 // ---- wait-timeout self test ---------------------------------------------------------
@@ -316,14 +348,36 @@ dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws);
   float* scores = reinterpret_cast<float*>(ws + f.idx_bytes);
   cudaStream_t s = (cudaStream_t)stream;
-  for (int r0 = 0; r0 < g.q_per_seq; r0 += f.chunk_rows) {
-    const int rc = std::min(f.chunk_rows, g.q_per_seq - r0);
+  const int r_end = g.row_begin + g.row_count;
+  for (int r0 = g.row_begin; r0 < r_end; r0 += f.chunk_rows) {
+    const int rc = std::min(f.chunk_rows, r_end - r0);
     st = launch_indexer(q_idx, w, k_idx, k_scale, g, scores, f.ld, r0, rc, s);
     if (st != DSA_OK) return st;
     st = launch_topk(scores, f.ld, g, r0, rc, k, idx, s);
     if (st != DSA_OK) return st;
   }
   return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, s);
+}
+
+dsa_status_t dsa_forward_noalloc(const void* q_idx, const float* w, const void* k_idx,
+                                 const float* k_scale, const void* q, const void* kv_cache,
+                                 const dsa_kv_desc_t* kv, const dsa_q_desc_t* qd, int32_t k,
+                                 float scale, int32_t* idx_out, void* out, float* lse,
+                                 dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  // The smallest workspace dsa_forward accepts: the indices (unless the caller
+  // receives them in idx_out) plus one score row per sequence.
+  const ForwardPlan f = plan_forward(g, k, idx_out == nullptr);
+  const size_t min_bytes = f.idx_bytes + align256((size_t)f.ld * 4 * g.batch);
+  if (min_bytes > kStaticScratchBytes) return DSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = static_scratch_address(&scratch);
+  if (st != DSA_OK) return st;
+  return dsa_forward(q_idx, w, k_idx, k_scale, q, kv_cache, kv, qd, k, scale, scratch,
+                     kStaticScratchBytes, idx_out, out, lse, stream);
 }
 
 dsa_status_t dsa_selftest_wait_timeout(dsa_stream_t stream) {
@@ -343,7 +397,7 @@ dsa_status_t dsa_indexer_scores(const void* q_idx, const float* w, const void* k
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
   if (ld < (int64_t)(g.max_ctx + kIdxTile - 1) / kIdxTile * kIdxTile || ld % 4 != 0)
     return DSA_ERR_INVALID_ARG;
-  return launch_indexer(q_idx, w, k_idx, k_scale, g, scores, ld, 0, g.q_per_seq,
+  return launch_indexer(q_idx, w, k_idx, k_scale, g, scores, ld, g.row_begin, g.row_count,
                         (cudaStream_t)stream);
 }
 
@@ -387,7 +441,7 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, const dsa_kv_desc_t* kv,
   if (!scores || !idx) return DSA_ERR_INVALID_ARG;
   if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (ld < g.max_ctx) return DSA_ERR_INVALID_ARG;
-  return launch_topk(scores, ld, g, 0, g.q_per_seq, k, idx, (cudaStream_t)stream);
+  return launch_topk(scores, ld, g, g.row_begin, g.row_count, k, idx, (cudaStream_t)stream);
 }
 
 }  // extern "C"

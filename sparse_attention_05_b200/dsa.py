@@ -65,6 +65,9 @@ SIGNATURES = {
     "dsa_forward": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.POINTER(KvDescC),
                                    ctypes.POINTER(QDescC), ctypes.c_int32, ctypes.c_float, _P,
                                    ctypes.c_size_t, _P, _P, _P, _P]),
+    "dsa_forward_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.POINTER(KvDescC),
+                                           ctypes.POINTER(QDescC), ctypes.c_int32, ctypes.c_float,
+                                           _P, _P, _P, _P]),
     "dsa_get_device_error": (ctypes.c_int, [_P]),
     "dsa_set_wait_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "dsa_selftest_wait_timeout": (ctypes.c_int, [_P]),
@@ -222,6 +225,25 @@ def dsa_forward(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_per_seq: 
                              _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k, float(scale),
                              _ptr(workspace), workspace.numel(), _ptr(idx_out), _ptr(out),
                              _ptr(lse), _stream(stream)), "dsa_forward")
+    return out, lse, idx_out
+
+
+def dsa_forward_noalloc(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_per_seq: int,
+                        k: int, scale: float, idx_out: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                        rows=None, stream=None):
+    """dsa_forward on the library's own fixed scratch array: the caller passes
+    inputs and outputs only (see include/dsa.h for the limits)."""
+    T = q.shape[0]
+    if out is None:
+        out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    _check(lib().dsa_forward_noalloc(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q),
+                                     _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k,
+                                     float(scale), _ptr(idx_out), _ptr(out), _ptr(lse),
+                                     _stream(stream)), "dsa_forward_noalloc")
     return out, lse, idx_out
 
 
