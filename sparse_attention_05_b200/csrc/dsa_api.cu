@@ -167,7 +167,10 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   p.G = std::min(4, row_count);
   p.groups_per_seq = (row_count + p.G - 1) / p.G;
   const int tiles = (g.max_ctx + kIdxTile - 1) / kIdxTile;
-  p.chunk_tiles = p.groups_per_seq == 1 ? 8 : tiles;
+  // decode: units of 32 tiles (4096 keys) spread sequences over all SMs while
+  // the next unit's query quantization hides behind the current unit's tiles;
+  // prefill: one unit per group of query rows (its whole causal row of tiles)
+  p.chunk_tiles = p.groups_per_seq == 1 ? 32 : tiles;
   p.chunks_per_group = (tiles + p.chunk_tiles - 1) / p.chunk_tiles;
   p.num_units = (int64_t)g.batch * p.groups_per_seq * p.chunks_per_group;
   p.timeout_ns = g_timeout_ns.load();
@@ -188,12 +191,9 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
-  CUtensorMap tm;
-  dsa_status_t st = make_tmap_2d(&tm, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDqk,
-                                 (uint64_t)g.num_q * kHeads, 64, 128);
-  if (st != DSA_OK) return st;
   MlaParams p{};
   p.kv = reinterpret_cast<const uint8_t*>(kv_cache);
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
   p.idx = idx;
   p.block_table = g.block_table;
   p.seqlens = g.seqlens;
@@ -224,7 +224,7 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, sparse_mla_kernel, p, tm));
+  return cuda_status(cudaLaunchKernelEx(&cfg, sparse_mla_kernel, p));
 }
 
 // ---- dsa_forward workspace plan --------------------------------------------------------

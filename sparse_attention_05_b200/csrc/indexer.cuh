@@ -15,12 +15,17 @@
 // from TMEM, so the H^I x L x L intermediate never reaches memory; one fp32
 // score per (row, key) is stored.
 //
-// Warp roles (256 threads):
-//   warp 0      TMA producer: key tiles (2 boxes of 64 rows x 128 B, 128-B swizzle)
+// Warp roles (384 threads):
+//   warp 0      producer: TMA key tiles (2 boxes of 64 rows x 128 B, 128-B swizzle)
+//               issued by lane 0, and the tile's 128 key scales staged by the
+//               whole warp with cp.async into a ring beside the key stages
 //   warp 1      TMEM allocation + single-thread tcgen05.mma issue
 //   warps 2-3   query quantizers: bf16 -> E4M3 rows in the canonical swizzled
 //               K-major layout, w*s_q per row (double-buffered per unit)
-//   warps 4-7   epilogue, thread = key (TMEM lane), 2 accumulator buffers
+//   warps 4-11  epilogue: two warpgroups, each owning one of the two TMEM
+//               accumulators (tiles alternate between them); thread = key lane
+// A stage of the ring is reused only after the MMA has read its keys and the
+// epilogue has read its scales.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -33,12 +38,13 @@ constexpr int kIdxHeads = 64;
 constexpr int kIdxDim = 128;
 constexpr int kIdxTile = 128;                      // keys per tile (MMA M)
 constexpr int kIdxStages = 8;
-constexpr int kIdxThreads = 256;
+constexpr int kIdxThreads = 384;
 constexpr int kIdxStageBytes = kIdxTile * kIdxDim;  // 16 KB of e4m3
 constexpr int kIdxQBufBytes = 4 * kIdxHeads * kIdxDim;  // G <= 4 rows x 64 heads x 128 B
 constexpr int kIdxSmemBytes =
     1024 /*align slack*/ + kIdxStages * kIdxStageBytes + 2 * kIdxQBufBytes +
-    2 * 4 * kIdxHeads * 4 /*wq*/ + 256 /*barriers etc*/;
+    2 * 4 * kIdxHeads * 4 /*wq*/ + kIdxStages * kIdxTile * 4 /*key scales*/ +
+    256 /*barriers etc*/;
 
 struct IndexerParams {
   const __nv_bfloat16* q_idx;  // [T][64][128]
@@ -103,7 +109,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint8_t* stages = smem;
   uint8_t* qbuf = stages + kIdxStages * kIdxStageBytes;
   float* wq = reinterpret_cast<float*>(qbuf + 2 * kIdxQBufBytes);  // [2][256]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(wq + 2 * 4 * kIdxHeads);
+  float* sscale = wq + 2 * 4 * kIdxHeads;                              // [stages][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sscale + kIdxStages * kIdxTile);
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + kIdxStages;
   uint64_t* tfull = bars + 2 * kIdxStages;
@@ -120,14 +127,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kIdxStages; ++s) {
-      mbar_init(smem_u32(&kfull[s]), 1);
-      mbar_init(smem_u32(&kempty[s]), 1);
+      mbar_init(smem_u32(&kfull[s]), 1 + 32);    // expect_tx arrival + 32 scale copiers
+      mbar_init(smem_u32(&kempty[s]), 1 + 128);  // MMA commit + the epilogue warpgroup
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);
       mbar_init(smem_u32(&tempty[i]), 128);
       mbar_init(smem_u32(&qfull[i]), 64);
-      mbar_init(smem_u32(&qempty[i]), 1 + 128);
+      mbar_init(smem_u32(&qempty[i]), 1 + 256);
     }
     mbar_init(smem_u32(mdone), 1);
     *abort_flag = 0;
@@ -146,38 +153,59 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   volatile int* no_abort = &drain_dummy;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tm_keys);
-      uint32_t it = 0;
-      for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
-        IdxUnit U;
-        if (!idx_unit(p, u, U)) continue;
-        const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
-        for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
-          const int st = it % kIdxStages;
-          if (!mbar_wait(smem_u32(&kempty[st]), ((it / kIdxStages) & 1) ^ 1, TO, abort_flag))
-            break;
-          const uint32_t bar = smem_u32(&kfull[st]);
-          mbar_arrive_expect_tx(bar, kIdxStageBytes);
+    // ------------------------------------------------------------ producer
+    if (lane == 0) prefetch_tmap(&tm_keys);
+    uint32_t it = 0;
+    for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+      IdxUnit U;
+      if (!idx_unit(p, u, U)) continue;
+      const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
+      bool ok = true;
+      for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
+        const int st = it % kIdxStages;
+        if (!warp_wait(smem_u32(&kempty[st]), ((it / kIdxStages) & 1) ^ 1, TO, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bar = smem_u32(&kfull[st]);
+        // cache rows of the tile's two 64-key halves (a half never straddles a page)
+        int64_t base[2] = {0, 0};
+        bool live[2] = {false, false};
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int s0 = kt * kIdxTile + h * 64;
-            int64_t row = 0;
-            if (s0 <= pos_max) {
-              bool ok;
-              row = idx_cache_row(p, U.b, s0, ok);
-              if (!ok) report_error(kErrBounds);
-            }
-            tma_load_2d(smem_u32(stages + st * kIdxStageBytes + h * 8192), &tm_keys, bar, 0,
-                        (int)row);
+        for (int h = 0; h < 2; ++h) {
+          const int s0 = kt * kIdxTile + h * 64;
+          if (s0 <= pos_max) {
+            bool rok;
+            base[h] = idx_cache_row(p, U.b, s0, rok);
+            live[h] = rok;
+            if (!rok && lane == 0) report_error(kErrBounds);
           }
         }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar, kIdxStageBytes);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(smem_u32(stages + st * kIdxStageBytes + h * 8192), &tm_keys, bar, 0,
+                        (int)base[h]);
+        }
+        // key scales: lane copies keys 4*lane .. 4*lane+3 of the tile
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int e = lane * 4 + v, h = e >> 6;
+          const int s = kt * kIdxTile + e;
+          const bool in = live[h] && s <= pos_max;
+          const float* src = p.k_scale + (in ? base[h] + (e & 63) : 0);
+          cp_async_4(smem_u32(sscale + st * kIdxTile + e), src, in ? 4u : 0u);
+        }
+        cp_async_mbar_arrive(bar);
       }
-      // Drain: the last stages' loads must land before the CTA may exit.
+      if (!ok) break;
+    }
+    // Drain: the last stages' copies must land before the CTA may exit.
+    if (lane == 0)
       for (uint32_t j = it > kIdxStages ? it - kIdxStages : 0; j < it; ++j)
         mbar_wait(smem_u32(&kfull[j % kIdxStages]), (j / kIdxStages) & 1, TO, no_abort);
-    }
+    cp_async_wait_all();
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -230,29 +258,50 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       if (!warp_wait(smem_u32(&qempty[qb]), ((un >> 1) & 1) ^ 1, TO, abort_flag)) break;
       uint8_t* qdst = qbuf + qb * kIdxQBufBytes;
       float* wdst = wq + qb * 4 * kIdxHeads;
-      for (int r = qw; r < N; r += 2) {
-        const int gi = r / kIdxHeads, j = r % kIdxHeads;
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-        float wj = 0.f;
-        if (gi < U.nrows) {
-          const int64_t t = (int64_t)U.b * p.q_per_seq + U.i0 + gi;
-          const uint2 raw = __ldg(reinterpret_cast<const uint2*>(
-              p.q_idx + (t * kIdxHeads + j) * kIdxDim + lane * 4));
-          x[0] = __uint_as_float(raw.x << 16);
-          x[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-          x[2] = __uint_as_float(raw.y << 16);
-          x[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-          wj = __ldg(p.w + t * kIdxHeads + j);
-        }
-        float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+      // A half-warp converts one 128-element row (8 elements = 16 B per lane);
+      // 8 rows per half-warp are loaded before any is used, so their global
+      // load latencies overlap. Rows r = base + 4 i of the batch.
+      const int half = lane >> 4, hl = lane & 15;
+      for (int base = qw * 2 + half; base < N; base += 32) {
+        uint4 raw[8];
+        float wj[8];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const float sq = __fdiv_rn(fmaxf(amax, 0x1p-120f), 448.0f);
-        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[0], sq), __fdiv_rn(x[1], sq));
-        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[2], sq), __fdiv_rn(x[3], sq));
-        *reinterpret_cast<uint32_t*>(qdst + sw128_offset(r, lane >> 2) + (lane & 3) * 4) =
-            lo | (hi << 16);
-        if (lane == 0) wdst[r] = wj * sq;
+        for (int i = 0; i < 8; ++i) {
+          const int r = base + 4 * i;
+          const int gi = r / kIdxHeads, j = r % kIdxHeads;
+          raw[i] = make_uint4(0u, 0u, 0u, 0u);
+          wj[i] = 0.f;
+          if (gi < U.nrows) {
+            const int64_t t = (int64_t)U.b * p.q_per_seq + U.i0 + gi;
+            raw[i] = __ldg(reinterpret_cast<const uint4*>(p.q_idx + (t * kIdxHeads + j) * kIdxDim) +
+                           hl);
+            wj[i] = __ldg(p.w + t * kIdxHeads + j);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = base + 4 * i;
+          const uint32_t wv[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+          float x[8];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            x[2 * c] = __uint_as_float(wv[c] << 16);
+            x[2 * c + 1] = __uint_as_float(wv[c] & 0xFFFF0000u);
+          }
+          float amax = 0.f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) amax = fmaxf(amax, fabsf(x[c]));
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          const float sq = __fdiv_rn(fmaxf(amax, 0x1p-120f), 448.0f);
+          uint32_t code[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            code[c] = cvt_e4m3x2(__fdiv_rn(x[2 * c], sq), __fdiv_rn(x[2 * c + 1], sq));
+          *reinterpret_cast<uint2*>(qdst + sw128_offset(r, hl >> 1) + (hl & 1) * 8) =
+              make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
+          if (hl == 0) wdst[r] = wj[i] * sq;
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(smem_u32(&qfull[qb]));
@@ -260,67 +309,74 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = tid - 128;           // key within the tile == TMEM lane
-    const int quad = warp - 4;         // TMEM lane quadrant of this warp
+    const int wg = (warp - 4) >> 2;    // warpgroup: owns TMEM accumulator `wg`
+    const int quad = warp & 3;         // TMEM lane quadrant of this warp
+    const int e = quad * 32 + lane;    // key within the tile == TMEM lane
     uint32_t it = 0, un = 0;
     for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
       IdxUnit U;
       if (!idx_unit(p, u, U)) {
         const int b = (int)(u / ((int64_t)p.groups_per_seq * p.chunks_per_group));
         const int sl = p.seqlens ? __ldg(p.seqlens + b) : p.max_ctx;
-        if (e == 0 && (sl < p.q_per_seq || sl > p.max_ctx)) report_error(kErrBounds);
+        if (wg == 0 && e == 0 && (sl < p.q_per_seq || sl > p.max_ctx)) report_error(kErrBounds);
         continue;
       }
       const int qb = un & 1;
       if (!warp_wait(smem_u32(&qfull[qb]), (un >> 1) & 1, TO, abort_flag)) break;
       const float* wrow = wq + qb * 4 * kIdxHeads;
       const int pos0 = U.seqlen - p.q_per_seq + U.i0;  // position of the group's first row
-      const int pos_max = pos0 + U.nrows - 1;
       bool ok = true;
       for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
-        const int ab = it & 1;
+        if ((int)(it & 1) != wg) continue;  // the other warpgroup's tile
+        const int st = it % kIdxStages;
         const int s = kt * kIdxTile + e;
-        float ks = 0.f;
-        if (s <= pos_max) {
-          bool rok;
-          const int64_t row = idx_cache_row(p, U.b, s, rok);
-          if (rok) ks = __ldg(p.k_scale + row);
+        if (!warp_wait(smem_u32(&kfull[st]), (it / kIdxStages) & 1, TO, abort_flag)) {
+          ok = false;
+          break;
         }
-        if (!warp_wait(smem_u32(&tfull[ab]), (it >> 1) & 1, TO, abort_flag)) {
+        const float ks = sscale[st * kIdxTile + e];
+        mbar_arrive(smem_u32(&kempty[st]));
+        if (!warp_wait(smem_u32(&tfull[wg]), (it >> 1) & 1, TO, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int gi = 0; gi < U.nrows; ++gi) {
-          float acc = 0.f;
+          // both 32-column loads in flight before one wait; four independent
+          // partial sums keep the FMA chains short
+          float v0[32], v1[32];
+          const uint32_t tcol =
+              tmem_base + ((uint32_t)(quad * 32) << 16) + wg * N + gi * kIdxHeads;
+          tmem_ld32(tcol, v0);
+          tmem_ld32(tcol + 32, v1);
+          tmem_wait_ld();
+          const float4* w4 = reinterpret_cast<const float4*>(wrow + gi * kIdxHeads);
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            float v[32];
-            tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + ab * N + gi * kIdxHeads +
-                          half * 32,
-                      v);
-            tmem_wait_ld();
-            const float4* w4 = reinterpret_cast<const float4*>(wrow + gi * kIdxHeads + half * 32);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const float4 ww = w4[q4];
-              acc = fmaf(ww.x, fmaxf(v[4 * q4 + 0], 0.f), acc);
-              acc = fmaf(ww.y, fmaxf(v[4 * q4 + 1], 0.f), acc);
-              acc = fmaf(ww.z, fmaxf(v[4 * q4 + 2], 0.f), acc);
-              acc = fmaf(ww.w, fmaxf(v[4 * q4 + 3], 0.f), acc);
-            }
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 wa = w4[q4], wb = w4[8 + q4];
+            a0 = fmaf(wa.x, fmaxf(v0[4 * q4 + 0], 0.f), a0);
+            a1 = fmaf(wa.y, fmaxf(v0[4 * q4 + 1], 0.f), a1);
+            a2 = fmaf(wa.z, fmaxf(v0[4 * q4 + 2], 0.f), a2);
+            a3 = fmaf(wa.w, fmaxf(v0[4 * q4 + 3], 0.f), a3);
+            a0 = fmaf(wb.x, fmaxf(v1[4 * q4 + 0], 0.f), a0);
+            a1 = fmaf(wb.y, fmaxf(v1[4 * q4 + 1], 0.f), a1);
+            a2 = fmaf(wb.z, fmaxf(v1[4 * q4 + 2], 0.f), a2);
+            a3 = fmaf(wb.w, fmaxf(v1[4 * q4 + 3], 0.f), a3);
           }
+          const float acc = (a0 + a1) + (a2 + a3);
           const float out = (s <= pos0 + gi) ? ks * acc : -INFINITY;
           const int64_t orow = (int64_t)U.b * p.row_count + (U.i0 - p.row_begin) + gi;
           p.scores[orow * p.ld + s] = out;
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&tempty[ab]));
+        mbar_arrive(smem_u32(&tempty[wg]));
       }
       if (!ok) break;
       mbar_arrive(smem_u32(&qempty[qb]));
       ++un;
     }
+    __syncwarp();
   }
 
   // ---------------------------------------------------------------- teardown
