@@ -166,16 +166,11 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   p.row_count = row_count;
   p.G = std::min(4, row_count);
   p.groups_per_seq = (row_count + p.G - 1) / p.G;
-  const int tiles = (g.max_ctx + kIdxTile - 1) / kIdxTile;
-  // decode: units of 32 tiles (4096 keys) spread sequences over all SMs while
-  // the next unit's query quantization hides behind the current unit's tiles;
-  // prefill: one unit per group of query rows (its whole causal row of tiles)
-  p.chunk_tiles = p.groups_per_seq == 1 ? 32 : tiles;
-  p.chunks_per_group = (tiles + p.chunk_tiles - 1) / p.chunk_tiles;
-  p.num_units = (int64_t)g.batch * p.groups_per_seq * p.chunks_per_group;
+  p.num_groups = g.batch * p.groups_per_seq;
   p.timeout_ns = g_timeout_ns.load();
-  if (p.num_units == 0) return DSA_OK;
-  const int grid = (int)std::min<int64_t>(p.num_units, num_sms());
+  // every CTA takes an equal share of all key tiles (at most one CTA per tile)
+  const int64_t max_tiles = (int64_t)p.num_groups * ((g.max_ctx + kIdxTile - 1) / kIdxTile);
+  const int grid = (int)std::min<int64_t>(max_tiles, num_sms());
   indexer_kernel<<<grid, kIdxThreads, kIdxSmemBytes, stream>>>(p, tm);
   return cuda_status(cudaGetLastError());
 }

@@ -7,8 +7,11 @@
 // E4M3 with s_q = max(amax, 2^-120) / 448, so that
 //   I_{t,s} = s_k[s] * sum_j (w_{t,j} s_q[t,j]) * ReLU(q_hat_{t,j} . k_hat_s).
 //
-// One persistent CTA per SM walks work units (sequence, group of G <= 4 query
-// rows, chunk of 128-key tiles). Per key tile the tensor core computes
+// One persistent CTA per SM. The work is the ordered list of 128-key tiles of
+// every (sequence, group of G <= 4 query rows); each CTA computes the total
+// from the sequence lengths itself and takes an exact equal share of that list
+// (sequences of very different lengths are balanced without any workspace).
+// A unit is the run of one group's tiles inside the share. Per key tile the tensor core computes
 //   D[key][(row, head)] = K_tile (128 x 128 e4m3) . Q_group^T (64G x 128 e4m3)
 // into TMEM (M = 128 keys in lanes, N = 64G columns). The epilogue applies the
 // ReLU, the w*s_q-weighted head sum, the key scale and the causal mask straight
@@ -44,7 +47,7 @@ constexpr int kIdxQBufBytes = 4 * kIdxHeads * kIdxDim;  // G <= 4 rows x 64 head
 constexpr int kIdxSmemBytes =
     1024 /*align slack*/ + kIdxStages * kIdxStageBytes + 2 * kIdxQBufBytes +
     2 * 4 * kIdxHeads * 4 /*wq*/ + kIdxStages * kIdxTile * 4 /*key scales*/ +
-    256 /*barriers etc*/;
+    256 /*barriers etc*/ + 512 /*share + scan scratch*/;
 
 struct IndexerParams {
   const __nv_bfloat16* q_idx;  // [T][64][128]
@@ -59,33 +62,123 @@ struct IndexerParams {
   int32_t row_begin, row_count;  // rows [row_begin, row_begin + row_count) of each sequence
   int32_t G;                     // query rows per MMA (N = 64 G)
   int32_t groups_per_seq;        // ceil(row_count / G)
-  int32_t chunk_tiles;           // key tiles per unit
-  int32_t chunks_per_group;
-  int64_t num_units;
+  int32_t num_groups;            // batch * groups_per_seq
   uint64_t timeout_ns;
 };
 
-// Everything a role needs to know about one work unit; all roles derive it
-// identically from the unit index and the (read-only) sequence lengths.
+// One unit: key tiles [kt0, kt1) of the group (sequence b, rows i0 .. i0+nrows-1).
 struct IdxUnit {
-  int b, i0, nrows, seqlen, kt0, kt1;  // key tiles [kt0, kt1)
+  int b, i0, nrows, seqlen, kt0, kt1;
 };
 
-__device__ __forceinline__ bool idx_unit(const IndexerParams& p, int64_t u, IdxUnit& U) {
-  const int64_t per_seq = (int64_t)p.groups_per_seq * p.chunks_per_group;
-  U.b = (int)(u / per_seq);
-  const int64_t rem = u - (int64_t)U.b * per_seq;
-  const int g = (int)(rem / p.chunks_per_group);
-  const int c = (int)(rem - (int64_t)g * p.chunks_per_group);
+// Tiles of group `grp` (0 when its sequence length is invalid) and its geometry.
+__device__ __forceinline__ int idx_group(const IndexerParams& p, int grp, IdxUnit& U) {
+  U.b = grp / p.groups_per_seq;
+  const int g = grp - U.b * p.groups_per_seq;
   U.seqlen = p.seqlens ? __ldg(p.seqlens + U.b) : p.max_ctx;
-  if (U.seqlen < p.q_per_seq || U.seqlen > p.max_ctx) return false;  // reported by the epilogue
+  if (U.seqlen < p.q_per_seq || U.seqlen > p.max_ctx) return 0;
   U.i0 = p.row_begin + g * p.G;
   U.nrows = min(p.G, p.row_begin + p.row_count - U.i0);
   const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
-  const int ntiles = pos_max / kIdxTile + 1;
-  U.kt0 = c * p.chunk_tiles;
-  U.kt1 = min(ntiles, U.kt0 + p.chunk_tiles);
-  return U.kt0 < U.kt1;
+  return pos_max / kIdxTile + 1;
+}
+
+// This CTA's share of the tile list: from (group gs, tile ts) to the exclusive
+// end (group ge, tile te); every role walks the same units with IdxCursor.
+struct IdxShare {
+  int gs, ts, ge, te;
+};
+struct IdxCursor {
+  int grp, kt;
+};
+__device__ __forceinline__ bool idx_next(const IndexerParams& p, const IdxShare& sh,
+                                         IdxCursor& c, IdxUnit& U) {
+  while (c.grp <= sh.ge && c.grp < p.num_groups) {
+    const int nt = idx_group(p, c.grp, U);
+    const int end = c.grp == sh.ge ? min(sh.te, nt) : nt;
+    if (c.kt < end) {
+      U.kt0 = c.kt;
+      U.kt1 = end;
+      ++c.grp;
+      c.kt = 0;
+      return true;
+    }
+    ++c.grp;
+    c.kt = 0;
+  }
+  return false;
+}
+
+// Work is balanced on a cost of (tiles + kIdxUnitCost) per group: a group's
+// query rows are quantized once per unit, which is worth about 16 tiles, so
+// many short causal groups (early prefill rows) weigh what they cost. A cost
+// position x within a group maps to the tile boundary max(0, x - kIdxUnitCost);
+// neighbouring shares apply the same map to their common boundary.
+constexpr int kIdxUnitCost = 16;
+
+// Block-wide: the exact share [W c / n, W (c+1) / n) of the total cost W.
+__device__ void idx_share(const IndexerParams& p, IdxShare* out, uint32_t* scratch) {
+  // scratch: [32] warp sums, [32] misc
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthreads = blockDim.x, nwarps = nthreads >> 5;
+  auto block_sum_scan = [&](long long v, long long& excl, long long& total) {
+    long long incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    long long* ws = reinterpret_cast<long long*>(scratch);
+    __syncthreads();
+    if (lane == 31) ws[warp] = incl;
+    __syncthreads();
+    long long before = 0, all = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      const long long x = ws[w];
+      if (w < warp) before += x;
+      all += x;
+    }
+    excl = before + incl - v;
+    total = all;
+  };
+  auto cost_of = [&](int grp, int& nt) -> long long {
+    IdxUnit U;
+    nt = grp < p.num_groups ? idx_group(p, grp, U) : 0;
+    return nt > 0 ? (long long)nt + kIdxUnitCost : 0;
+  };
+  // pass 1: total cost
+  long long W = 0;
+  for (int base = 0; base < p.num_groups; base += nthreads) {
+    int nt;
+    const long long cost = cost_of(base + tid, nt);
+    long long excl, tot;
+    block_sum_scan(cost, excl, tot);
+    W += tot;
+  }
+  const long long lo = W * blockIdx.x / gridDim.x, hi = W * (blockIdx.x + 1) / gridDim.x;
+  if (tid == 0) *out = IdxShare{p.num_groups, 0, -1, 0};  // empty unless found below
+  __syncthreads();
+  if (lo >= hi) return;
+  // pass 2: locate the groups holding cost positions lo and hi - 1
+  long long run = 0;
+  for (int base = 0; base < p.num_groups; base += nthreads) {
+    const int grp = base + tid;
+    int nt;
+    const long long cost = cost_of(grp, nt);
+    long long excl, tot;
+    block_sum_scan(cost, excl, tot);
+    const long long a = run + excl, e = a + cost;  // cost positions [a, e) belong to grp
+    if (cost > 0 && a <= lo && lo < e) {
+      out->gs = grp;
+      out->ts = (int)max(0ll, lo - a - kIdxUnitCost);
+    }
+    if (cost > 0 && a < hi && hi <= e) {
+      out->ge = grp;
+      out->te = (int)max(0ll, hi - a - kIdxUnitCost);
+    }
+    run += tot;
+  }
+  __syncthreads();
 }
 
 // Cache row of logical token s of sequence b (s must be < seqlen for paged).
@@ -120,6 +213,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint64_t* mdone = qempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  IdxShare* share = reinterpret_cast<IdxShare*>(tmem_holder + 4);
+  uint32_t* scan_scratch = reinterpret_cast<uint32_t*>(share + 1) + 4;  // 8-B aligned, 32 x i64
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = kIdxHeads * p.G;
@@ -147,6 +242,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  idx_share(p, share, scan_scratch);  // ends with a barrier
+  const IdxShare sh = *share;
   const uint32_t tmem_base = *tmem_holder;
   const uint64_t TO = p.timeout_ns;
   int drain_dummy = 0;
@@ -156,9 +253,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) prefetch_tmap(&tm_keys);
     uint32_t it = 0;
-    for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
-      IdxUnit U;
-      if (!idx_unit(p, u, U)) continue;
+    IdxCursor cur{sh.gs, sh.ts};
+    IdxUnit U;
+    while (!*abort_flag && idx_next(p, sh, cur, U)) {
       const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
       bool ok = true;
       for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
@@ -212,9 +309,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = instr_desc(0 /*e4m3*/, 0, 0, 128, N);
       uint32_t it = 0, un = 0;
-      for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
-        IdxUnit U;
-        if (!idx_unit(p, u, U)) continue;
+      IdxCursor cur{sh.gs, sh.ts};
+      IdxUnit U;
+      while (!*abort_flag && idx_next(p, sh, cur, U)) {
         const int qb = un & 1;
         if (!mbar_wait(smem_u32(&qfull[qb]), (un >> 1) & 1, TO, abort_flag)) break;
         const uint32_t qaddr = smem_u32(qbuf + qb * kIdxQBufBytes);
@@ -251,9 +348,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // ------------------------------------------------------------ query quantizers
     const int qw = warp - 2;  // 0..1
     uint32_t un = 0;
-    for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
-      IdxUnit U;
-      if (!idx_unit(p, u, U)) continue;
+    IdxCursor cur{sh.gs, sh.ts};
+    IdxUnit U;
+    while (!*abort_flag && idx_next(p, sh, cur, U)) {
       const int qb = un & 1;
       if (!warp_wait(smem_u32(&qempty[qb]), ((un >> 1) & 1) ^ 1, TO, abort_flag)) break;
       uint8_t* qdst = qbuf + qb * kIdxQBufBytes;
@@ -313,14 +410,15 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const int quad = warp & 3;         // TMEM lane quadrant of this warp
     const int e = quad * 32 + lane;    // key within the tile == TMEM lane
     uint32_t it = 0, un = 0;
-    for (int64_t u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
-      IdxUnit U;
-      if (!idx_unit(p, u, U)) {
-        const int b = (int)(u / ((int64_t)p.groups_per_seq * p.chunks_per_group));
+    if (blockIdx.x == 0 && wg == 0) {  // sequences whose length cannot hold their rows
+      for (int b = e; b < p.batch; b += 128) {
         const int sl = p.seqlens ? __ldg(p.seqlens + b) : p.max_ctx;
-        if (wg == 0 && e == 0 && (sl < p.q_per_seq || sl > p.max_ctx)) report_error(kErrBounds);
-        continue;
+        if (sl < p.q_per_seq || sl > p.max_ctx) report_error(kErrBounds);
       }
+    }
+    IdxCursor cur{sh.gs, sh.ts};
+    IdxUnit U;
+    while (!*abort_flag && idx_next(p, sh, cur, U)) {
       const int qb = un & 1;
       if (!warp_wait(smem_u32(&qfull[qb]), (un >> 1) & 1, TO, abort_flag)) break;
       const float* wrow = wq + qb * 4 * kIdxHeads;

@@ -210,14 +210,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
       if (mbar_wait(smem_u32(qfull), 0, TO, abort_flag)) {
         tc_fence_after();
         // Issue S_j (needs block j landed and P_{j-3}.V issued: its score buffer
-        // is reused) and P_i.V (needs P_i written) in order of readiness.
+        // is reused) and P_i.V (needs P_i written) in order of readiness; the
+        // barriers are tested without suspending, so neither waits on the other.
         int js = 0, jp = 0;
         uint64_t t_last = globaltimer_ns();
         uint32_t spins = 0;
         while (jp < nblk && !*abort_flag) {
           bool progressed = false;
           if (js < nblk && js < jp + kMlaSBufs &&
-              mbar_try_wait(smem_u32(&kvfull[js % kMlaStages]), (js / kMlaStages) & 1)) {
+              mbar_test_wait(smem_u32(&kvfull[js % kMlaStages]), (js / kMlaStages) & 1)) {
             fence_proxy_async_smem();  // cp.async writes -> tensor-core reads
             tc_fence_after();
             const uint32_t ka = smem_u32(sKV + (js % kMlaStages) * kMlaStageBytes);
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
             ++js;
             progressed = true;
           }
-          if (jp < js && mbar_try_wait(smem_u32(&pfull[jp % kMlaSBufs]), (jp / kMlaSBufs) & 1)) {
+          if (jp < js && mbar_test_wait(smem_u32(&pfull[jp % kMlaSBufs]), (jp / kMlaSBufs) & 1)) {
             tc_fence_after();
             const uint32_t va = smem_u32(sKV + (jp % kMlaStages) * kMlaStageBytes);
 #pragma unroll
