@@ -113,7 +113,8 @@ DSA_API dsa_status_t dsa_indexer_scores(const void* q_idx, const float* w, const
 
 /* Fine-grained token selection (report §1 and §2.1: S_t = Top-k(I_{t,:})).
  *  scores fp32 [batch * row_count][ld] as dsa_indexer_scores writes it: the
- *         row of query t is read on [0, pos(t)] only.
+ *         row of query t is read on [0, pos(t)] only. 16-byte aligned, ld >= max_ctx
+ *         and a multiple of 4.
  *  idx    int32 [T][k] out: the k highest-scoring positions of row t in
  *         ascending order; equal scores keep the lower position (-0.0 == +0.0);
  *         when pos(t) + 1 <= k all visible positions are selected and the rest

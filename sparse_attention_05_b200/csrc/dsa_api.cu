@@ -435,7 +435,7 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, const dsa_kv_desc_t* kv,
   if (st != DSA_OK) return st;
   if (!scores || !idx) return DSA_ERR_INVALID_ARG;
   if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
-  if (ld < g.max_ctx) return DSA_ERR_INVALID_ARG;
+  if (ld < g.max_ctx || ld % 4 != 0 || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
   return launch_topk(scores, ld, g, g.row_begin, g.row_count, k, idx, (cudaStream_t)stream);
 }
 

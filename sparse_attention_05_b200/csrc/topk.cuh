@@ -2,16 +2,22 @@
 // lightning-indexer scores among the visible keys (DeepSeek-V3.2-Exp technical
 // report, zh translation, §1 "Architecture" and §2.1: S_t = Top-k(I_{t,:})).
 //
-// One CTA of 1024 threads per row, radix select on an order-preserving 32-bit
-// key of each fp32 score:
-//   pass 1..3  histograms of key bits [31:21], [20:10], [9:0] restricted to the
+// One CTA of 1024 threads per row. Scores are compared through an
+// order-preserving 32-bit key (-0.0 maps to +0.0). The exact selection is a
+// radix select:
+//   find_kth   histograms of key bits [31:21], [20:10], [9:0] restricted to the
 //              prefix found so far -> the exact k-th largest key tau and the
 //              number r of keys equal to tau that belong to the selection;
-//   compaction one ordered sweep: a key > tau is selected, a key == tau is
+//   compact    one ordered sweep: a key > tau is selected, a key == tau is
 //              selected while fewer than r equal keys precede it, so equal
 //              scores keep the lower position and the output is ascending.
-// Rows of up to kTopkCacheElems scores stay in shared memory across passes;
-// longer rows are re-read from global memory (L2) on every pass.
+// Long rows (more than 4k keys) first shrink to a candidate list: a fixed
+// strided sample of 2048 scores gives a threshold that lies, with a wide
+// margin, below the k-th score; one coalesced sweep keeps the keys at or above
+// it in position order, and the exact selection runs on the candidates. The
+// candidates hold the k largest keys whenever there are at least k of them, so
+// the result is exact; if the sample misjudged (fewer than k candidates, or
+// more than the buffer holds) the row falls back to the exact full-row path.
 #pragma once
 
 #include "ptx.cuh"
@@ -20,7 +26,9 @@ namespace dsa {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkCacheElems = 40 * 1024;                     // 160 KB row cache
-constexpr int kTopkSmemBytes = kTopkCacheElems * 4 + 2048 * 4 + 64 * 4;
+constexpr int kTopkCandCap = kTopkCacheElems / 2;              // candidates: key + position
+constexpr int kTopkSample = 2048;
+constexpr int kTopkSmemBytes = kTopkCacheElems * 4 + 2048 * 4 + 64 * 4 + kTopkSample * 4;
 
 struct TopkParams {
   const float* scores;
@@ -69,38 +77,14 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   return warp_tot[warp] + incl - v;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  float* cache = reinterpret_cast<float*>(smem_raw);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw + kTopkCacheElems * 4);
-  uint32_t* misc = hist + 2048;  // [0..31] warp totals, [32] total, [33] digit, [34] remaining
-
-  const int b = blockIdx.x / p.row_count;
-  const int i = p.row_begin + blockIdx.x % p.row_count;
-  const int64_t t = (int64_t)b * p.q_per_seq + i;
+// The k-th largest key among elements [0, n) (k <= n) and how many keys equal to
+// it belong to the top k. misc: [0..31] warp totals, [32] total, [33..34] result.
+template <class KeyAt>
+__device__ void find_kth(int n, uint32_t k, KeyAt key_at, uint32_t* hist, uint32_t* misc,
+                         uint32_t& tau, uint32_t& r_eq) {
   const int tid = threadIdx.x;
-  int32_t* out = p.idx + t * p.k;
-
-  const int seqlen = p.seqlens ? p.seqlens[b] : p.max_ctx;
-  if (seqlen < p.q_per_seq || seqlen > p.max_ctx) {
-    if (tid == 0) report_error(kErrBounds);
-    for (int j = tid; j < p.k; j += kTopkThreads) out[j] = -1;
-    return;
-  }
-  const int n = seqlen - p.q_per_seq + i + 1;  // visible keys 0..pos
-  if (n <= p.k) {
-    for (int j = tid; j < p.k; j += kTopkThreads) out[j] = j < n ? j : -1;
-    return;
-  }
-
-  const float* row = p.scores + (int64_t)(blockIdx.x) * p.ld;
-  const bool cached = n <= kTopkCacheElems;
   const int n_iter = (n + kTopkThreads - 1) / kTopkThreads;
-
-  uint32_t prefix = 0;       // key bits fixed so far
-  uint32_t prefix_mask = 0;  // which bits of the key are fixed
-  uint32_t remaining = p.k;  // how many of the k still lie at or below the prefix
-
+  uint32_t prefix = 0, prefix_mask = 0, remaining = k;
   const int shifts[3] = {21, 10, 0};
   const int widths[3] = {11, 11, 10};
 #pragma unroll 1
@@ -114,14 +98,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
       const int e = it * kTopkThreads + tid;
       uint32_t digit = 0xFFFFFFFFu;
       if (e < n) {
-        float x;
-        if (pass == 0) {
-          x = row[e];
-          if (cached) cache[e] = x;
-        } else {
-          x = cached ? cache[e] : row[e];
-        }
-        const uint32_t key = score_key(x);
+        const uint32_t key = key_at(e, pass);
         if ((key & prefix_mask) == prefix) digit = (key >> shift) & (nbins - 1);
       }
       const uint32_t peers = __match_any_sync(0xffffffffu, digit);
@@ -129,8 +106,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
         atomicAdd(&hist[digit], __popc(peers));
     }
     __syncthreads();
-    // Find the bin holding the remaining-th largest key: threads walk the bins
-    // from the top, two bins per thread (bins 2047-2*tid and 2046-2*tid).
+    // the bin holding the remaining-th largest key: bins walked from the top,
+    // two per thread (2047 - 2 tid, 2046 - 2 tid)
     const int hi_bin = 2047 - 2 * tid, lo_bin = 2046 - 2 * tid;
     const uint32_t c_hi = hi_bin < (int)nbins ? hist[hi_bin] : 0;
     const uint32_t c_lo = lo_bin < (int)nbins ? hist[lo_bin] : 0;
@@ -149,10 +126,15 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
     prefix_mask |= (nbins - 1) << shift;
     __syncthreads();
   }
-  const uint32_t tau = prefix;      // exact key of the k-th largest score
-  const uint32_t r_eq = remaining;  // keys == tau to take, lowest positions first
+  tau = prefix;
+  r_eq = remaining;
+}
 
-  // Ordered compaction: each thread owns 8 consecutive positions per sweep.
+// Ordered compaction of the top k: positions pos_at(e) must increase with e.
+template <class KeyAt, class PosAt>
+__device__ void compact_topk(int n, uint32_t tau, uint32_t r_eq, KeyAt key_at, PosAt pos_at,
+                             int32_t* out, uint32_t* misc) {
+  const int tid = threadIdx.x;
   uint32_t gt_run = 0, eq_run = 0;  // selected-above / equal counts before this sweep
   const int per_sweep = kTopkThreads * 8;
 #pragma unroll 1
@@ -165,7 +147,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
       const int e = e0 + u;
       keys[u] = 0;
       if (e < n) {
-        keys[u] = score_key(cached ? cache[e] : row[e]);
+        keys[u] = key_at(e, 3);
         n_gt += keys[u] > tau;
         n_eq += keys[u] == tau;
       }
@@ -179,10 +161,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
       const int e = e0 + u;
       if (e >= n) break;
       if (keys[u] > tau) {
-        out[gt_b + min(eq_b, r_eq)] = e;
+        out[gt_b + min(eq_b, r_eq)] = pos_at(e);
         ++gt_b;
       } else if (keys[u] == tau) {
-        if (eq_b < r_eq) out[gt_b + eq_b] = e;
+        if (eq_b < r_eq) out[gt_b + eq_b] = pos_at(e);
         ++eq_b;
       }
     }
@@ -190,6 +172,119 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
     eq_run += sweep_tot & 0xFFFFu;
     __syncthreads();  // misc reused by the next sweep's scan
   }
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  float* cache = reinterpret_cast<float*>(smem_raw);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw + kTopkCacheElems * 4);
+  uint32_t* misc = hist + 2048;  // [0..31] warp totals, [32] total, [33..35] results
+  uint32_t* sample = misc + 64;  // [kTopkSample]
+  uint32_t* cand_key = reinterpret_cast<uint32_t*>(cache);      // [kTopkCandCap]
+  int32_t* cand_pos = reinterpret_cast<int32_t*>(cache) + kTopkCandCap;
+
+  const int b = blockIdx.x / p.row_count;
+  const int i = p.row_begin + blockIdx.x % p.row_count;
+  const int64_t t = (int64_t)b * p.q_per_seq + i;
+  const int tid = threadIdx.x;
+  int32_t* out = p.idx + t * p.k;
+
+  const int seqlen = p.seqlens ? p.seqlens[b] : p.max_ctx;
+  if (seqlen < p.q_per_seq || seqlen > p.max_ctx) {
+    if (tid == 0) report_error(kErrBounds);
+    for (int j = tid; j < p.k; j += kTopkThreads) out[j] = -1;
+    return;
+  }
+  const int n = seqlen - p.q_per_seq + i + 1;  // visible keys 0..pos
+  const uint32_t k = (uint32_t)p.k;
+  if (n <= p.k) {
+    for (int j = tid; j < p.k; j += kTopkThreads) out[j] = j < n ? j : -1;
+    return;
+  }
+  const float* row = p.scores + (int64_t)(blockIdx.x) * p.ld;
+  uint32_t tau, r_eq;
+
+  if (n > 4 * p.k) {
+    // ---- candidate filter ------------------------------------------------------
+    // strided sample -> threshold with a wide safety margin below the k-th key
+    for (int s = tid; s < kTopkSample; s += kTopkThreads)
+      sample[s] = score_key(row[(int64_t)s * n / kTopkSample]);
+    __syncthreads();
+    const float frac = (float)p.k / (float)n;
+    const float expect = frac * kTopkSample;
+    uint32_t r = (uint32_t)(expect + 4.0f * sqrtf(expect) + 16.0f);
+    r = min(r, (uint32_t)kTopkSample);
+    uint32_t tau_low, unused;
+    find_kth(kTopkSample, r, [&](int e, int) { return sample[e]; }, hist, misc, tau_low, unused);
+    // keep keys >= tau_low in position order (4 consecutive keys per thread)
+    uint32_t m_run = 0;
+    bool overflow = false;
+#pragma unroll 1
+    for (int base = 0; base < n; base += 4 * kTopkThreads) {
+      const int e0 = base + 4 * tid;
+      uint32_t kk[4];
+      uint32_t c = 0;
+      if (e0 + 3 < n) {  // rows start 16-B aligned (ld is a multiple of 4)
+        const float4 v = *reinterpret_cast<const float4*>(row + e0);
+        kk[0] = score_key(v.x);
+        kk[1] = score_key(v.y);
+        kk[2] = score_key(v.z);
+        kk[3] = score_key(v.w);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) kk[u] = (e0 + u < n) ? score_key(row[e0 + u]) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) c += (e0 + u < n) && kk[u] >= tau_low;
+      const uint32_t excl = block_exclusive_scan(c, misc, misc + 32);
+      const uint32_t tot = misc[32];
+      uint32_t w = m_run + excl;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if ((e0 + u < n) && kk[u] >= tau_low) {
+          if (w < (uint32_t)kTopkCandCap) {
+            cand_key[w] = kk[u];
+            cand_pos[w] = e0 + u;
+          }
+          ++w;
+        }
+      }
+      m_run += tot;
+      overflow = m_run > (uint32_t)kTopkCandCap;
+      __syncthreads();
+      if (overflow) break;
+    }
+    if (!overflow && m_run >= k) {
+      const int m = (int)m_run;
+      find_kth(m, k, [&](int e, int) { return cand_key[e]; }, hist, misc, tau, r_eq);
+      compact_topk(m, tau, r_eq, [&](int e, int) { return cand_key[e]; },
+                   [&](int e) { return cand_pos[e]; }, out, misc);
+      return;
+    }
+    // the sample misjudged this row: exact selection over the whole row
+    __syncthreads();
+    find_kth(n, k, [&](int e, int) { return score_key(row[e]); }, hist, misc, tau, r_eq);
+    compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(row[e]); },
+                 [&](int e) { return e; }, out, misc);
+    return;
+  }
+
+  // ---- short rows: cached in shared memory across the passes ---------------------
+  // (n <= 4k <= 8192 <= kTopkCacheElems)
+  find_kth(n, k,
+           [&](int e, int pass) {
+             float x;
+             if (pass == 0) {
+               x = row[e];
+               cache[e] = x;
+             } else {
+               x = cache[e];
+             }
+             return score_key(x);
+           },
+           hist, misc, tau, r_eq);
+  compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(cache[e]); },
+               [&](int e) { return e; }, out, misc);
 }
 
 }  // namespace dsa

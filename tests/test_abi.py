@@ -104,6 +104,8 @@ def test_host_argument_checks_without_gpu(lib):
     assert L.dsa_topk(fake, 512, by(kv), by(bad_q), 2048, fake, None) == 1
     # row window outside the sequence
     assert L.dsa_topk(fake, 512, by(kv), by(dsa.QDescC(2, 1, 1, 0)), 2048, fake, None) == 1
+    # top-k score rows must be 16-byte aligned
+    assert L.dsa_topk(fake, 514, by(kv), by(q), 2048, fake, None) == 1
     # ld below max_ctx rounded to 128
     assert L.dsa_indexer_scores(fake, fake, fake, fake, by(kv), by(q), fake, 500, None) == 1
     # misaligned pointer
