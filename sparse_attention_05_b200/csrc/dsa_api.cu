@@ -20,7 +20,7 @@ using namespace dsa;
 
 namespace {
 
-constexpr int kDIdx = 128, kHeads = 128, kDqk = 576, kMaxK = 2048;
+constexpr int kDIdx = 128, kMaxK = 2048;
 
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 
@@ -186,6 +186,11 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  // the latent cache as [cache_rows][576] bf16, gathered 64 dims of one row per box row
+  CUtensorMap tm;
+  dsa_status_t st = make_tmap_2d(&tm, kv_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMlaDqk,
+                                 (uint64_t)g.cache_rows, 64, 1);
+  if (st != DSA_OK) return st;
   MlaParams p{};
   p.kv = reinterpret_cast<const uint8_t*>(kv_cache);
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -219,7 +224,7 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, sparse_mla_kernel, p));
+  return cuda_status(cudaLaunchKernelEx(&cfg, sparse_mla_kernel, p, tm));
 }
 
 // ---- dsa_forward workspace plan --------------------------------------------------------

@@ -9,35 +9,44 @@
 //
 // Design: one 2-CTA cluster per query token. O (128 heads x 512 fp32) would
 // fill all of one SM's tensor memory, so CTA r of the pair owns value dims
-// [256 r, 256 r + 256) and contracts QK^T over its own slice of the key dims:
-//   r = 0: key dims [0, 256)    (= its value dims)
-//   r = 1: key dims [256, 576)  (its value dims + the 64 rope dims)
-// Every gathered latent byte is loaded by exactly one CTA. The two partial
+// [256 r, 256 r + 256) and contracts QK^T over its own 288 of the 576 key dims:
+// its value dims plus half of the 64 rope dims ([512 + 32 r, 544 + 32 r)).
+// Each CTA gathers its 256 value dims and the 64 rope dims of a row. The two partial
 // score tiles are swapped through distributed shared memory and added
 // (a + b == b + a, so both CTAs hold bit-identical scores and take identical
 // softmax decisions); each CTA then runs O_r += P . V[:, its value dims].
 //
-// Tensor memory: O (256 columns), three score buffers of 32 columns (P, as
-// bf16 pairs, later overwrites the first 16 columns of its scores) and this
-// CTA's slice of Q (128 or 160 columns, two bf16 per column): Q and P are read
-// by the tensor core straight from tensor memory, which leaves shared memory to
-// a deep gather ring and the exchange buffers.
+// Tensor memory: O (256 columns), this CTA's Q slice (144 columns, two bf16
+// per column) and two score buffers of 48 columns (P, as bf16 pairs, later
+// overwrites the first 24 columns of its scores). Q and P are read by the
+// tensor core straight from tensor memory, which leaves shared memory to the
+// gather ring and the exchange buffers. Every tcgen05.mma costs about the same
+// issue time up to N = 128, so blocks are as wide as the budget allows.
 //
-// Pipeline, per block of 32 selected keys:
-//   producers (warps 0-1)  resolve cache rows one block ahead and gather the
-//                          rows' slice with cp.async (zero fill for entries
-//                          outside [0, pos]) into a 6-stage 128-B-swizzled ring;
-//                          completion arrives asynchronously on the stage barrier
-//   MMA (warp 10)          S_j = Q . K_j^T (M=128 heads, N=32, K=256|320, Q from
-//                          TMEM) and O += P_j . V_j (M=128, N=256, K=32, P from
+// Pipeline, per block of 48 selected keys:
+//   resolver (warp 1)      turns selected indices into cache rows (-1 outside
+//                          [0, pos]) and valid-key bits, four blocks at a time,
+//                          for the whole row up front, into a shared table
+//   gather (warps 0, 11-15) each SM's TMA unit moves only about one 128-B
+//                          gathered row per ~20 cycles, and cp.async throughput
+//                          grows with the number of issuing threads, so both
+//                          are used side by side: warp 0 gathers rows 0-23 of
+//                          the block with TMA tile::gather4 (four rows x 64
+//                          dims per copy, 128-B swizzle, zero fill for row -1),
+//                          warps 11-15 copy rows 24-47 in 16-B cp.async pieces
+//                          (zero fill for row -1) into the same swizzled
+//                          4-stage ring; both complete the stage barrier
+//   MMA (warp 10)          S_j = Q . K_j^T (M=128 heads, N=48, K=288, Q from
+//                          TMEM) and O += P_j . V_j (M=128, N=256, K=48, P from
 //                          TMEM, V MN-major), each issued as soon as it is ready
-//   softmax (warps 2-9)    thread = (head, half of the block's keys). Block j+1's
-//                          partial scores go to the peer before block j's softmax
-//                          runs; four exchange buffers mean the peer can only
-//                          overwrite a buffer after a chain of data dependencies
-//                          through this CTA's later sends, so no handshake is
-//                          needed. Online softmax in base 2 with a lazy rescale
-//                          of O (only when the running max grows by more than 8).
+//   softmax (warps 2-9)    thread = (head, half of the block's keys). Block j's
+//                          partial scores go to the peer as soon as S_j lands,
+//                          while the tensor core already computes S_{j+1}; three
+//                          exchange buffers mean the peer can only overwrite a
+//                          buffer after a chain of data dependencies through this
+//                          CTA's later sends, so no handshake is needed. Online
+//                          softmax in base 2 with a lazy rescale of O (only when
+//                          the running max grows by more than 8).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -49,24 +58,33 @@ namespace dsa {
 constexpr int kMlaHeads = 128;
 constexpr int kMlaDqk = 576;
 constexpr int kMlaDv = 512;
-constexpr int kMlaBlk = 32;                   // keys per block
+constexpr int kMlaBlk = 48;                   // keys per block
 constexpr int kMlaHalf = kMlaBlk / 2;         // keys per softmax thread
-constexpr int kMlaStages = 6;                 // gather ring
-constexpr int kMlaSBufs = 3;                  // TMEM score / probability buffers
-constexpr int kMlaXBufs = 4;                  // exchange buffers
-constexpr int kMlaThreads = 352;              // 2 producer, 8 softmax, 1 MMA warp
+constexpr int kMlaStages = 4;                 // gather ring
+constexpr int kMlaSBufs = 2;                  // TMEM score / probability buffers
+constexpr int kMlaXBufs = 3;                  // exchange buffers
+constexpr int kMlaThreads = 512;              // TMA, resolver, 8 softmax, MMA, 5 cp.async warps
 constexpr int kMlaMmaWarp = 10;
-constexpr int kMlaKChunk = kMlaBlk * 128;     // 64-dim column chunk of a block: 4 KB
-constexpr int kMlaStageBytes = 5 * kMlaKChunk;
-constexpr int kMlaXRow = 36;                  // floats per exchange row (32 + pad)
+constexpr int kMlaCpWarp0 = 11;               // first cp.async warp
+constexpr int kMlaCpThreads = 160;
+constexpr int kMlaTmaRows = 24;               // rows of a block gathered by TMA
+constexpr int kMlaKChunk = kMlaBlk * 128;     // 64-dim column chunk of a block: 6 KB
+constexpr int kMlaStageBytes = 5 * kMlaKChunk;  // 4 value chunks + the 64 rope dims
+constexpr int kMlaQCols = 144;                // TMEM columns of the Q slice
+constexpr int kMlaMaxK = 2048;
+constexpr int kMlaResolve = 4 * kMlaBlk;      // keys the resolver handles per step
+constexpr int kMlaMaxSteps = (kMlaMaxK + kMlaResolve - 1) / kMlaResolve;  // 11
+constexpr int kMlaRowCap = kMlaMaxSteps * kMlaResolve;                   // 2112
+constexpr int kMlaMaskWords = kMlaRowCap / 32 + 2;
+constexpr int kMlaXRow = 52;                  // floats per exchange row (48 + pad)
 constexpr int kMlaXBytes = kMlaHeads * kMlaXRow * 4;
 constexpr int kMlaXPayload = kMlaHeads * kMlaBlk * 4;  // bytes the peer sends per block
 constexpr int kMlaSmemBytes = 1024 + kMlaStages * kMlaStageBytes + kMlaXBufs * kMlaXBytes +
-                              kMlaStages * kMlaBlk * 4 /*rows*/ + 8 * 4 /*masks*/ +
-                              2 * 2 * kMlaHeads * 4 /*max swap*/ + 32 * 8 /*barriers*/ + 16;
+                              kMlaRowCap * 4 /*rows*/ + kMlaMaskWords * 4 /*valid bits*/ +
+                              2 * 2 * kMlaHeads * 4 /*max swap*/ + 40 * 8 /*barriers*/ + 16;
 constexpr uint32_t kMlaTmemCols = 512;
-constexpr uint32_t kMlaTmemS = 256;           // score buffers at 256, 288, 320
-constexpr uint32_t kMlaTmemQ = 352;           // Q slice: 128 or 160 columns
+constexpr uint32_t kMlaTmemS = 256;           // score buffers in 64-column slots at 256, 320
+constexpr uint32_t kMlaTmemQ = 368;           // Q slice: columns [368, 512)
 
 struct MlaParams {
   const uint8_t* kv;           // latent cache rows of 1152 B
@@ -84,24 +102,26 @@ struct MlaParams {
   uint64_t timeout_ns;
 };
 
-__global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid_constant__ MlaParams p) {
+__global__ void __launch_bounds__(kMlaThreads, 1)
+    sparse_mla_kernel(const __grid_constant__ MlaParams p, const __grid_constant__ CUtensorMap tm_kv) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sKV = smem;
-  uint8_t* sX = sKV + kMlaStages * kMlaStageBytes;                      // [4][128][36] f32
-  int32_t* sRow = reinterpret_cast<int32_t*>(sX + kMlaXBufs * kMlaXBytes);   // [6][32]
-  uint32_t* sMask = reinterpret_cast<uint32_t*>(sRow + kMlaStages * kMlaBlk);  // [8]
-  float* sRed = reinterpret_cast<float*>(sMask + 8);                  // [2][2][128]
+  uint8_t* sX = sKV + kMlaStages * kMlaStageBytes;                      // [3][128][52] f32
+  int32_t* sRow = reinterpret_cast<int32_t*>(sX + kMlaXBufs * kMlaXBytes);   // [2112]
+  uint32_t* sBits = reinterpret_cast<uint32_t*>(sRow + kMlaRowCap);   // valid-key bits
+  float* sRed = reinterpret_cast<float*>(sBits + kMlaMaskWords);      // [2][2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRed + 2 * 2 * kMlaHeads);
-  uint64_t* kvfull = bars + 0;     // [6] stage landed + mask published
-  uint64_t* kvempty = bars + 6;    // [6] O += P V of the stage's block done
-  uint64_t* sfull = bars + 12;     // [3] S in score buffer
-  uint64_t* pfull = bars + 15;     // [3] P written over S
-  uint64_t* xfull = bars + 18;     // [4] peer's partial scores arrived
-  uint64_t* qfull = bars + 22;     // Q stored in TMEM
-  uint64_t* mdone = bars + 23;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24);
+  uint64_t* kvfull = bars;                     // [stages] stage landed
+  uint64_t* kvempty = kvfull + kMlaStages;      // [stages] O += P V of the stage's block done
+  uint64_t* sfull = kvempty + kMlaStages;       // [2] S in score buffer
+  uint64_t* pfull = sfull + kMlaSBufs;          // [2] P written over S
+  uint64_t* xfull = pfull + kMlaSBufs;          // [3] peer's partial scores arrived
+  uint64_t* qfull = xfull + kMlaXBufs;          // Q stored in TMEM
+  uint64_t* mdone = qfull + 1;
+  uint64_t* rready = mdone + 1;                 // [11] resolver step done
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(rready + kMlaMaxSteps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -111,13 +131,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
   const int b = (int)(local / p.row_count);
   const int qi = p.row_begin + (int)(local - (int64_t)b * p.row_count);
   const int64_t t = (int64_t)b * p.q_per_seq + qi;  // global query row
-  const int nchunk = 4 + (int)rank;      // 64-dim column chunks of this CTA's key slice
-  const int d0 = 256 * (int)rank;        // first key dim of the slice (also first value dim)
+  const int d0 = 256 * (int)rank;        // first value dim (and first key dim) of this CTA
+  const int r0 = 512 + 32 * (int)rank;   // this CTA's quarter of the rope dims
   const int nblk = (p.k + kMlaBlk - 1) / kMlaBlk;
 
   if (tid == 0) {
     for (int i = 0; i < kMlaStages; ++i) {
-      mbar_init(smem_u32(&kvfull[i]), 64 + 1);  // 64 async cp.async arrivals + mask writer
+      // the TMA warp's expect_tx arrival (+ its bytes) and one asynchronous
+      // arrival per cp.async thread once its copies have landed
+      mbar_init(smem_u32(&kvfull[i]), 1 + kMlaCpThreads);
       mbar_init(smem_u32(&kvempty[i]), 1);
     }
     for (int i = 0; i < kMlaSBufs; ++i) {
@@ -127,6 +149,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
     for (int i = 0; i < kMlaXBufs; ++i) mbar_init(smem_u32(&xfull[i]), 1);  // + peer's bytes
     mbar_init(smem_u32(qfull), 256);
     mbar_init(smem_u32(mdone), 1);
+    for (int i = 0; i < kMlaMaxSteps; ++i) mbar_init(smem_u32(&rready[i]), 1);
     *abort_flag = 0;
     fence_mbarrier_init_cluster();
   }
@@ -141,7 +164,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
   const uint32_t tmem_base = *tmem_holder;
   const uint32_t tO = tmem_base;
   const uint32_t tQ = tmem_base + kMlaTmemQ;
-  auto tS = [&](int j) { return tmem_base + kMlaTmemS + 32u * (uint32_t)(j % kMlaSBufs); };
+  auto tS = [&](int j) { return tmem_base + kMlaTmemS + 64u * (uint32_t)(j % kMlaSBufs); };
   const uint64_t TO = p.timeout_ns;
   int drain_dummy = 0;
   volatile int* no_abort = &drain_dummy;
@@ -151,57 +174,99 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
   const bool seq_ok = seqlen >= p.q_per_seq && seqlen <= p.max_ctx;
   const int pos = seqlen - p.q_per_seq + qi;
 
-  if (warp < 2) {
-    // ------------------------------------------------------------ gather producers
-    const int nch16 = nchunk * 8;  // 16-byte chunks per row slice
-    // Cache rows of block j into sRow[j % 6] (-1: outside [0, pos], zero-filled)
-    // and its valid-key mask into sMask[j & 7].
-    auto rows_for = [&](int j) {
-      if (warp == 0) {
-        const int e = j * kMlaBlk + lane;
-        const int s = e < p.k ? __ldg(p.idx + t * p.k + e) : -1;
+  if (warp == 1) {
+    // ------------------------------------------------------------ row resolver
+    // Step c covers keys [192 c, 192 c + 192): lane l takes keys 192 c + 32 i + l,
+    // so all six index loads (and then all six block-table loads) are in flight
+    // together. No slot is ever reused, so the resolver never waits.
+    const int nsteps = (nblk + 3) / 4;
+    for (int c = 0; c < nsteps; ++c) {
+      int sel[6], pg[6];
+#pragma unroll
+      for (int i = 0; i < 6; ++i) {
+        const int e = c * kMlaResolve + 32 * i + lane;
+        sel[i] = e < p.k ? __ldg(p.idx + t * p.k + e) : -1;
+        if (!(seq_ok && sel[i] >= 0 && sel[i] <= pos)) sel[i] = -1;
+      }
+      if (p.paged) {
+#pragma unroll
+        for (int i = 0; i < 6; ++i)
+          pg[i] = sel[i] >= 0 ? __ldg(p.block_table + (int64_t)b * p.max_pages + sel[i] / p.page_size)
+                              : -1;
+      }
+#pragma unroll
+      for (int i = 0; i < 6; ++i) {
         int row = -1;
-        if (seq_ok && s >= 0 && s <= pos) {
+        if (sel[i] >= 0) {
           if (!p.paged) {
-            row = b * p.max_ctx + s;
+            row = b * p.max_ctx + sel[i];
+          } else if (pg[i] >= 0 && pg[i] < p.num_pages) {
+            row = pg[i] * p.page_size + sel[i] % p.page_size;
           } else {
-            const int pg = __ldg(p.block_table + (int64_t)b * p.max_pages + s / p.page_size);
-            if (pg >= 0 && pg < p.num_pages) row = pg * p.page_size + s % p.page_size;
-            else report_error(kErrBounds);
+            report_error(kErrBounds);
           }
         }
-        sRow[(j % kMlaStages) * kMlaBlk + lane] = row;
+        sRow[c * kMlaResolve + 32 * i + lane] = row;
         const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
-        if (lane == 0) sMask[j & 7] = m;
+        if (lane == 0) sBits[c * 6 + i] = m;
       }
-    };
-    if (nblk > 0) rows_for(0);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&rready[c]));  // releases the rows and bits
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ TMA gather
+    if (lane == 0) prefetch_tmap(&tm_kv);
+    int issued = 0;
     for (int j = 0; j < nblk; ++j) {
       const int st = j % kMlaStages;
-      // The stage is free once O += P V of block j-6 has finished. Both producer
-      // warps decide together (neither is left behind in a barrier when a wait
-      // gives up); the barrier also publishes sRow[st].
-      const bool ok = warp_wait(smem_u32(&kvempty[st]), ((j / kMlaStages) & 1) ^ 1, TO, abort_flag);
-      if (!named_barrier_and(1, 64, ok)) break;
-      {
-        // two threads per key row: chunks c = (tid & 1), (tid & 1) + 2, ...
-        const int kr = tid >> 1;
-        const int row = sRow[st * kMlaBlk + kr];
-        const uint8_t* src = p.kv + (row >= 0 ? (int64_t)row * (kMlaDqk * 2) : 0) + d0 * 2;
-        const uint32_t dst = smem_u32(sKV + st * kMlaStageBytes) + kr * 128;
-        const uint32_t nbytes = row >= 0 ? 16u : 0u;
-        for (int c = tid & 1; c < nch16; c += 2)
-          cp_async_16(dst + (c >> 3) * kMlaKChunk + (((c & 7) ^ (kr & 7)) << 4), src + c * 16,
-                      nbytes);
+      // the stage is free once O += P V of block j-4 has finished
+      bool ok = warp_wait(smem_u32(&kvempty[st]), ((j / kMlaStages) & 1) ^ 1, TO, abort_flag);
+      if (ok && (j & 3) == 0) ok = warp_wait(smem_u32(&rready[j >> 2]), 0, TO, abort_flag);
+      if (!ok) break;
+      const uint32_t bar = smem_u32(&kvfull[st]);
+      if (lane == 0) mbar_arrive_expect_tx(bar, kMlaTmaRows * 5 * 128);
+      __syncwarp();
+      if (lane < kMlaTmaRows / 4) {
+        // rows 4 lane .. 4 lane + 3 of the block: value dims [d0, d0 + 256) in
+        // four 64-dim chunks, then the 64 rope dims
+        const int4 r = *reinterpret_cast<const int4*>(sRow + j * kMlaBlk + 4 * lane);
+        const uint32_t dst = smem_u32(sKV + st * kMlaStageBytes) + lane * 4 * 128;
+#pragma unroll
+        for (int cb = 0; cb < 5; ++cb)
+          tma_gather4(dst + cb * kMlaKChunk, &tm_kv, bar, cb < 4 ? d0 + 64 * cb : kMlaDv, r.x,
+                      r.y, r.z, r.w);
       }
-      // this thread's copies arrive on kvfull[st] when they land (no waiting here)
+      issued = j + 1;
+    }
+    // on an early exit, let the copies still in flight land before the CTA can leave
+    for (int jj = issued > kMlaStages ? issued - kMlaStages : 0; jj < issued; ++jj)
+      warp_wait(smem_u32(&kvfull[jj % kMlaStages]), (jj / kMlaStages) & 1, TO, no_abort);
+  } else if (warp >= kMlaCpWarp0) {
+    // ------------------------------------------------------------ cp.async gather
+    // rows [24, 48) of each block: 40 pieces of 16 B per row (value dims
+    // [d0, d0 + 256) into chunks 0-3, the 64 rope dims into chunk 4), six per
+    // thread; a warp's 32 consecutive pieces lie in one or two rows
+    const int ct = tid - kMlaCpWarp0 * 32;
+    for (int j = 0; j < nblk; ++j) {
+      const int st = j % kMlaStages;
+      bool ok = warp_wait(smem_u32(&kvempty[st]), ((j / kMlaStages) & 1) ^ 1, TO, abort_flag);
+      if (ok && (j & 3) == 0) ok = warp_wait(smem_u32(&rready[j >> 2]), 0, TO, abort_flag);
+      if (!ok) break;
+      const uint32_t sbase = smem_u32(sKV + st * kMlaStageBytes);
+#pragma unroll
+      for (int i = 0; i < (kMlaBlk - kMlaTmaRows) * 40 / kMlaCpThreads; ++i) {
+        const int ci = ct + i * kMlaCpThreads;
+        const int kr = kMlaTmaRows + ci / 40, c = ci % 40;
+        const int row = sRow[j * kMlaBlk + kr];
+        const int dim = c < 32 ? d0 + 8 * c : kMlaDv + 8 * (c - 32);
+        cp_async_16(sbase + (c >> 3) * kMlaKChunk + kr * 128 + (((c & 7) ^ (kr & 7)) << 4),
+                    p.kv + (row >= 0 ? (int64_t)row * (kMlaDqk * 2) + dim * 2 : 0),
+                    row >= 0 ? 16u : 0u);
+      }
+      // arrives on the stage barrier once this thread's copies have landed
       cp_async_mbar_arrive(smem_u32(&kvfull[st]));
-      // the block's mask word (written one block earlier) is released by its writer
-      if (tid == 0) mbar_arrive(smem_u32(&kvfull[st]));
-      if (j + 1 < nblk) rows_for(j + 1);
     }
     cp_async_wait_all();
-    __syncwarp();
   } else if (warp == kMlaMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -209,7 +274,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
       const uint32_t idesc_pv = instr_desc(1, 0, 1 /*V is MN-major*/, 128, 256);
       if (mbar_wait(smem_u32(qfull), 0, TO, abort_flag)) {
         tc_fence_after();
-        // Issue S_j (needs block j landed and P_{j-3}.V issued: its score buffer
+        // Issue S_j (needs block j landed and P_{j-2}.V issued: its score buffer
         // is reused) and P_i.V (needs P_i written) in order of readiness; the
         // barriers are tested without suspending, so neither waits on the other.
         int js = 0, jp = 0;
@@ -219,12 +284,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
           bool progressed = false;
           if (js < nblk && js < jp + kMlaSBufs &&
               mbar_test_wait(smem_u32(&kvfull[js % kMlaStages]), (js / kMlaStages) & 1)) {
-            fence_proxy_async_smem();  // cp.async writes -> tensor-core reads
             tc_fence_after();
+            fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor-core reads
             const uint32_t ka = smem_u32(sKV + (js % kMlaStages) * kMlaStageBytes);
-            for (int kk = 0; kk < nchunk * 4; ++kk) {
+            for (int kk = 0; kk < kMlaQCols / 8; ++kk) {  // 16 value + 2 rope K-steps
+              // rope: this CTA's 32 dims sit at bytes [64 r, 64 r + 64) of the row
+              const int kb = kk < 16 ? (kk & 3) : (kk & 3) + 2 * (int)rank;
               const uint64_t bd =
-                  smem_desc_sw128(ka + (kk >> 2) * kMlaKChunk + (kk & 3) * 32, 16, 1024);
+                  smem_desc_sw128(ka + (kk >> 2) * kMlaKChunk + kb * 32, 16, 1024);
               mma_bf16_ts(tS(js), tQ + kk * 8, bd, idesc_s, kk > 0 ? 1u : 0u);
             }
             mma_commit(smem_u32(&sfull[js % kMlaSBufs]));
@@ -267,37 +334,30 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
     const uint32_t xrow_off = (uint32_t)h * (kMlaXRow * 4) + (uint32_t)k0 * 4;
     const bool announcer = (hf == 0 && h == 0);  // arms this CTA's xfull phases
 
-    // Q slice -> TMEM (row h = lane h): this half stores columns
-    // [hf * qcols/2, (hf + 1) * qcols/2), two bf16 per column.
+    // Q slice -> TMEM (row h = lane h, two bf16 per column): column c holds
+    // dims d0 + 2c (c < 128) or r0 + 2(c - 128); this half stores columns
+    // [72 hf, 72 hf + 72) in steps of 8 columns (16 dims, 32 bytes).
     {
-      const int qcols = 32 * nchunk;
-      const int c0 = hf * (qcols / 2);
-      const uint4* src = reinterpret_cast<const uint4*>(
-          p.q + (t * kMlaHeads + h) * kMlaDqk + d0 + 2 * c0);
-      for (int c = 0; c < qcols / 2; c += 16) {  // 16 columns = 32 dims = 64 B per step
-        uint32_t w[16];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 x = __ldg(src + (c / 4) + v);
-          w[4 * v] = x.x;
-          w[4 * v + 1] = x.y;
-          w[4 * v + 2] = x.z;
-          w[4 * v + 3] = x.w;
-        }
-        tmem_st8(tQ + c0 + c + lane_off, w);
-        tmem_st8(tQ + c0 + c + 8 + lane_off, w + 8);
+      const __nv_bfloat16* qrow = p.q + (t * kMlaHeads + h) * kMlaDqk;
+      for (int c = hf * (kMlaQCols / 2); c < (hf + 1) * (kMlaQCols / 2); c += 8) {
+        const int dim = c < 128 ? d0 + 2 * c : r0 + 2 * (c - 128);
+        const uint4* src = reinterpret_cast<const uint4*>(qrow + dim);
+        const uint4 x0 = __ldg(src), x1 = __ldg(src + 1);
+        const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        tmem_st8(tQ + c + lane_off, w);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(qfull));
     }
 
-    auto load_s = [&](int j, float* v) {  // this thread's 16 scores of block j
+    auto load_s = [&](int j, float* v) {  // this thread's 24 scores of block j
       tmem_ld16(tS(j) + k0 + lane_off, v);
+      tmem_ld8(tS(j) + k0 + 16 + lane_off, v + 16);
       tmem_wait_ld();
     };
     auto send = [&](int j, const float* v) {  // partial scores of block j -> peer
-      const uint32_t xb = (uint32_t)(j & (kMlaXBufs - 1));
+      const uint32_t xb = (uint32_t)(j % kMlaXBufs);
       const uint32_t dst = x_peer + xb * kMlaXBytes + xrow_off;
       const uint32_t bar = xfull_peer0 + xb * 8;
 #pragma unroll
@@ -306,39 +366,23 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
     };
 
     float m_used = -INFINITY, l = 0.f;
-    float cur[kMlaHalf], nxt[kMlaHalf];
-#pragma unroll
-    for (int i = 0; i < kMlaHalf; ++i) cur[i] = nxt[i] = 0.f;
+    float cur[kMlaHalf];
     bool ok = true;
-    // prologue: block 0's partial goes out first
-    if (nblk > 0) {
-      if (announcer) mbar_arrive_expect_tx(smem_u32(&xfull[0]), kMlaXPayload);
-      ok = warp_wait(smem_u32(&sfull[0]), 0, TO, abort_flag);
+    for (int j = 0; j < nblk; ++j) {
+      const int xb = j % kMlaXBufs;
+      // (A) block j: own partial scores from TMEM, sent to the peer. The exchange
+      // buffer was last used for block j-3, which both CTAs consumed before
+      // sending blocks j-2 and j-1 that the other has waited on since.
+      if (announcer) mbar_arrive_expect_tx(smem_u32(&xfull[xb]), kMlaXPayload);
+      if (ok) ok = warp_wait(smem_u32(&sfull[j % kMlaSBufs]), (j / kMlaSBufs) & 1, TO, abort_flag);
       if (ok) {
         tc_fence_after();
-        load_s(0, cur);
-        send(0, cur);
+        load_s(j, cur);
+        send(j, cur);
       }
-    }
-    for (int j = 0; j < nblk; ++j) {
-      const int xb = j & (kMlaXBufs - 1);
-      // (A) block j+1: scores from TMEM, partial sent to the peer. Its buffer
-      // was last used for block j-3, which this CTA consumed three blocks ago,
-      // before sending blocks j-1 and j that the peer has waited on since.
-      if (ok && j + 1 < nblk) {
-        if (announcer)
-          mbar_arrive_expect_tx(smem_u32(&xfull[(j + 1) & (kMlaXBufs - 1)]), kMlaXPayload);
-        ok = warp_wait(smem_u32(&sfull[(j + 1) % kMlaSBufs]), ((j + 1) / kMlaSBufs) & 1, TO,
-                       abort_flag);
-        if (ok) {
-          tc_fence_after();
-          load_s(j + 1, nxt);
-          send(j + 1, nxt);
-        }
-      }
-      // (B) block j: full scores = own partial + the peer's
+      // (B) full scores = own partial + the peer's
       float mhalf = -INFINITY;
-      if (ok) ok = warp_wait<true>(smem_u32(&xfull[xb]), (j >> 2) & 1, TO, abort_flag);
+      if (ok) ok = warp_wait<true>(smem_u32(&xfull[xb]), (j / kMlaXBufs) & 1, TO, abort_flag);
       if (ok) {
         const float* xr = reinterpret_cast<const float*>(sX + xb * kMlaXBytes + xrow_off);
 #pragma unroll
@@ -352,7 +396,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
         ok = warp_wait(smem_u32(&kvfull[j % kMlaStages]), (j / kMlaStages) & 1, TO, abort_flag);
       }
       if (ok) {
-        const uint32_t mask = (sMask[j & 7] >> k0) & 0xFFFFu;
+        const int b0 = j * kMlaBlk + k0;  // this half's 24 valid-key bits
+        const uint64_t w2 = ((uint64_t)sBits[(b0 >> 5) + 1] << 32) | sBits[b0 >> 5];
+        const uint32_t mask = (uint32_t)(w2 >> (b0 & 31)) & 0xFFFFFFu;
 #pragma unroll
         for (int i = 0; i < kMlaHalf; ++i) {
           cur[i] = ((mask >> i) & 1u) ? cur[i] * p.scale_log2 : -INFINITY;
@@ -404,14 +450,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(const __grid
           pk[i] = pack_bf16x2(p0, p1);
         }
         l += lsum;
-        // P_j over S_j: packed columns [8 hf, 8 hf + 8) of score buffer j
+        // P_j over S_j: packed columns [12 hf, 12 hf + 12) of score buffer j
         tmem_st8(tS(j) + hf * (kMlaHalf / 2) + lane_off, pk);
+        tmem_st4(tS(j) + hf * (kMlaHalf / 2) + 8 + lane_off, pk + 8);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(smem_u32(&pfull[j % kMlaSBufs]));
       }
-#pragma unroll
-      for (int i = 0; i < kMlaHalf; ++i) cur[i] = nxt[i];
     }
     // epilogue: every P.V product has finished once the last one has (in order)
     if (ok && nblk > 0)
