@@ -16,12 +16,13 @@
 // (a + b == b + a, so both CTAs hold bit-identical scores and take identical
 // softmax decisions); each CTA then runs O_r += P . V[:, its value dims].
 //
-// Tensor memory: O (256 columns), this CTA's Q slice (144 columns, two bf16
-// per column) and two score buffers of 48 columns (P, as bf16 pairs, later
-// overwrites the first 24 columns of its scores). Q and P are read by the
-// tensor core straight from tensor memory, which leaves shared memory to the
-// gather ring and the exchange buffers. Every tcgen05.mma costs about the same
-// issue time up to N = 128, so blocks are as wide as the budget allows.
+// Tensor memory: O (256 columns), three score buffers of 48 columns (P, as
+// bf16 pairs, later overwrites the first 24 columns of its scores) and the
+// first 224 of this CTA's 288 Q dims (112 columns, two bf16 per column); the
+// other 64 Q dims (the last 32 value dims and this CTA's 32 rope dims) sit in
+// one 128-B-swizzled shared-memory chunk. A tcgen05.mma of M = 128, K = 16
+// takes about the same time for any N up to 256, so blocks are as wide as the
+// budget allows and the tensor core never waits for a free score buffer.
 //
 // Pipeline, per block of 48 selected keys:
 //   resolver (warp 1)      turns selected indices into cache rows (-1 outside
@@ -39,14 +40,16 @@
 //   MMA (warp 10)          S_j = Q . K_j^T (M=128 heads, N=48, K=288, Q from
 //                          TMEM) and O += P_j . V_j (M=128, N=256, K=48, P from
 //                          TMEM, V MN-major), each issued as soon as it is ready
-//   softmax (warps 2-9)    thread = (head, half of the block's keys). Block j's
-//                          partial scores go to the peer as soon as S_j lands,
-//                          while the tensor core already computes S_{j+1}; three
-//                          exchange buffers mean the peer can only overwrite a
-//                          buffer after a chain of data dependencies through this
-//                          CTA's later sends, so no handshake is needed. Online
-//                          softmax in base 2 with a lazy rescale of O (only when
-//                          the running max grows by more than 8).
+//   softmax (warps 2-9)    thread = (head, half of the block's keys). The
+//                          exchange is the scarcest resource (distributed shared
+//                          memory moves ~20 GB/s per SM), so it never idles:
+//                          block j+1's partial scores are sent to the peer
+//                          before block j's softmax runs. The peer's partials
+//                          land in a two-buffer ring; after consuming a buffer
+//                          this CTA re-arms it and hands the peer a credit (a
+//                          remote mbarrier arrival) for the block two ahead.
+//                          Online softmax in base 2 with a lazy rescale of O
+//                          (only when the running max grows by more than 8).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -61,8 +64,8 @@ constexpr int kMlaDv = 512;
 constexpr int kMlaBlk = 48;                   // keys per block
 constexpr int kMlaHalf = kMlaBlk / 2;         // keys per softmax thread
 constexpr int kMlaStages = 4;                 // gather ring
-constexpr int kMlaSBufs = 2;                  // TMEM score / probability buffers
-constexpr int kMlaXBufs = 3;                  // exchange buffers
+constexpr int kMlaSBufs = 3;                  // TMEM score / probability buffers
+constexpr int kMlaXBufs = 2;                  // exchange ring (credit based)
 constexpr int kMlaThreads = 512;              // TMA, resolver, 8 softmax, MMA, 5 cp.async warps
 constexpr int kMlaMmaWarp = 10;
 constexpr int kMlaCpWarp0 = 11;               // first cp.async warp
@@ -70,7 +73,10 @@ constexpr int kMlaCpThreads = 160;
 constexpr int kMlaTmaRows = 24;               // rows of a block gathered by TMA
 constexpr int kMlaKChunk = kMlaBlk * 128;     // 64-dim column chunk of a block: 6 KB
 constexpr int kMlaStageBytes = 5 * kMlaKChunk;  // 4 value chunks + the 64 rope dims
-constexpr int kMlaQCols = 144;                // TMEM columns of the Q slice
+constexpr int kMlaKSteps = 18;                // K = 16 steps over this CTA's 288 dims
+constexpr int kMlaQCols = 112;                // TMEM columns of Q: dims [0, 224) of the slice
+constexpr int kMlaQTmemSteps = kMlaQCols / 8; // K-steps whose A operand is in TMEM (14)
+constexpr int kMlaQSmemBytes = kMlaHeads * 128;  // last 64 Q dims, one swizzled chunk
 constexpr int kMlaMaxK = 2048;
 constexpr int kMlaResolve = 4 * kMlaBlk;      // keys the resolver handles per step
 constexpr int kMlaMaxSteps = (kMlaMaxK + kMlaResolve - 1) / kMlaResolve;  // 11
@@ -79,12 +85,16 @@ constexpr int kMlaMaskWords = kMlaRowCap / 32 + 2;
 constexpr int kMlaXRow = 52;                  // floats per exchange row (48 + pad)
 constexpr int kMlaXBytes = kMlaHeads * kMlaXRow * 4;
 constexpr int kMlaXPayload = kMlaHeads * kMlaBlk * 4;  // bytes the peer sends per block
-constexpr int kMlaSmemBytes = 1024 + kMlaStages * kMlaStageBytes + kMlaXBufs * kMlaXBytes +
-                              kMlaRowCap * 4 /*rows*/ + kMlaMaskWords * 4 /*valid bits*/ +
-                              2 * 2 * kMlaHeads * 4 /*max swap*/ + 40 * 8 /*barriers*/ + 16;
+constexpr int kMlaSmemBytes = 1024 + kMlaStages * kMlaStageBytes + kMlaQSmemBytes +
+                              kMlaXBufs * kMlaXBytes + kMlaRowCap * 4 /*rows*/ +
+                              kMlaMaskWords * 4 /*valid bits*/ + 2 * 2 * kMlaHeads * 4 /*max swap*/ +
+                              40 * 8 /*barriers*/ + 16;
+static_assert(kMlaSmemBytes <= 232448, "sparse MLA shared memory exceeds the per-CTA limit");
 constexpr uint32_t kMlaTmemCols = 512;
-constexpr uint32_t kMlaTmemS = 256;           // score buffers in 64-column slots at 256, 320
-constexpr uint32_t kMlaTmemQ = 368;           // Q slice: columns [368, 512)
+constexpr uint32_t kMlaTmemS = 256;           // score buffers at columns 256, 304, 352
+constexpr uint32_t kMlaTmemQ = 400;           // Q: columns [400, 512)
+static_assert(kMlaTmemS + kMlaSBufs * kMlaBlk <= kMlaTmemQ && kMlaTmemQ + kMlaQCols <= kMlaTmemCols,
+              "sparse MLA tensor-memory plan overlaps");
 
 struct MlaParams {
   const uint8_t* kv;           // latent cache rows of 1152 B
@@ -108,7 +118,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sKV = smem;
-  uint8_t* sX = sKV + kMlaStages * kMlaStageBytes;                      // [3][128][52] f32
+  uint8_t* sQ = sKV + kMlaStages * kMlaStageBytes;                      // [128][128 B] swizzled
+  uint8_t* sX = sQ + kMlaQSmemBytes;                                    // [2][128][52] f32
   int32_t* sRow = reinterpret_cast<int32_t*>(sX + kMlaXBufs * kMlaXBytes);   // [2112]
   uint32_t* sBits = reinterpret_cast<uint32_t*>(sRow + kMlaRowCap);   // valid-key bits
   float* sRed = reinterpret_cast<float*>(sBits + kMlaMaskWords);      // [2][2][128]
@@ -117,8 +128,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   uint64_t* kvempty = kvfull + kMlaStages;      // [stages] O += P V of the stage's block done
   uint64_t* sfull = kvempty + kMlaStages;       // [2] S in score buffer
   uint64_t* pfull = sfull + kMlaSBufs;          // [2] P written over S
-  uint64_t* xfull = pfull + kMlaSBufs;          // [3] peer's partial scores arrived
-  uint64_t* qfull = xfull + kMlaXBufs;          // Q stored in TMEM
+  uint64_t* xfull = pfull + kMlaSBufs;          // [2] peer's partial scores arrived
+  uint64_t* xfree = xfull + kMlaXBufs;          // [2] the peer consumed this CTA's send (credit)
+  uint64_t* qfull = xfree + kMlaXBufs;          // Q stored in TMEM and shared memory
   uint64_t* mdone = qfull + 1;
   uint64_t* rready = mdone + 1;                 // [11] resolver step done
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(rready + kMlaMaxSteps);
@@ -146,11 +158,18 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       mbar_init(smem_u32(&sfull[i]), 1);
       mbar_init(smem_u32(&pfull[i]), 256);
     }
-    for (int i = 0; i < kMlaXBufs; ++i) mbar_init(smem_u32(&xfull[i]), 1);  // + peer's bytes
+    for (int i = 0; i < kMlaXBufs; ++i) {
+      mbar_init(smem_u32(&xfull[i]), 1);  // + the peer's bytes
+      mbar_init(smem_u32(&xfree[i]), 1);  // one remote arrival from the peer
+    }
     mbar_init(smem_u32(qfull), 256);
     mbar_init(smem_u32(mdone), 1);
     for (int i = 0; i < kMlaMaxSteps; ++i) mbar_init(smem_u32(&rready[i]), 1);
     *abort_flag = 0;
+    // the first two blocks' exchange buffers start free: arm them before the
+    // peer may send (later blocks are armed when their buffer is consumed)
+    for (int i = 0; i < kMlaXBufs && i < nblk; ++i)
+      mbar_arrive_expect_tx(smem_u32(&xfull[i]), kMlaXPayload);
     fence_mbarrier_init_cluster();
   }
   if (warp == kMlaMmaWarp) {
@@ -164,7 +183,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const uint32_t tmem_base = *tmem_holder;
   const uint32_t tO = tmem_base;
   const uint32_t tQ = tmem_base + kMlaTmemQ;
-  auto tS = [&](int j) { return tmem_base + kMlaTmemS + 64u * (uint32_t)(j % kMlaSBufs); };
+  auto tS = [&](int j) {
+    return tmem_base + kMlaTmemS + (uint32_t)kMlaBlk * (uint32_t)(j % kMlaSBufs);
+  };
   const uint64_t TO = p.timeout_ns;
   int drain_dummy = 0;
   volatile int* no_abort = &drain_dummy;
@@ -274,47 +295,52 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       const uint32_t idesc_pv = instr_desc(1, 0, 1 /*V is MN-major*/, 128, 256);
       if (mbar_wait(smem_u32(qfull), 0, TO, abort_flag)) {
         tc_fence_after();
-        // Issue S_j (needs block j landed and P_{j-2}.V issued: its score buffer
-        // is reused) and P_i.V (needs P_i written) in order of readiness; the
-        // barriers are tested without suspending, so neither waits on the other.
-        int js = 0, jp = 0;
-        uint64_t t_last = globaltimer_ns();
-        uint32_t spins = 0;
-        while (jp < nblk && !*abort_flag) {
-          bool progressed = false;
-          if (js < nblk && js < jp + kMlaSBufs &&
-              mbar_test_wait(smem_u32(&kvfull[js % kMlaStages]), (js / kMlaStages) & 1)) {
-            tc_fence_after();
-            fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor-core reads
-            const uint32_t ka = smem_u32(sKV + (js % kMlaStages) * kMlaStageBytes);
-            for (int kk = 0; kk < kMlaQCols / 8; ++kk) {  // 16 value + 2 rope K-steps
-              // rope: this CTA's 32 dims sit at bytes [64 r, 64 r + 64) of the row
-              const int kb = kk < 16 ? (kk & 3) : (kk & 3) + 2 * (int)rank;
-              const uint64_t bd =
-                  smem_desc_sw128(ka + (kk >> 2) * kMlaKChunk + kb * 32, 16, 1024);
+        auto issue_s = [&](int js) {  // S_js = Q . K_js^T into score buffer js % 3
+          tc_fence_after();
+          fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor-core reads
+          const uint32_t ka = smem_u32(sKV + (js % kMlaStages) * kMlaStageBytes);
+          for (int kk = 0; kk < kMlaKSteps; ++kk) {  // 16 value + 2 rope K-steps
+            // rope: this CTA's 32 dims sit at bytes [64 r, 64 r + 64) of the row
+            const int kb = kk < 16 ? (kk & 3) : (kk & 3) + 2 * (int)rank;
+            const uint64_t bd = smem_desc_sw128(ka + (kk >> 2) * kMlaKChunk + kb * 32, 16, 1024);
+            if (kk < kMlaQTmemSteps) {
               mma_bf16_ts(tS(js), tQ + kk * 8, bd, idesc_s, kk > 0 ? 1u : 0u);
+            } else {  // Q's last 64 dims: 32-B K-steps of the shared-memory chunk
+              const uint64_t qd =
+                  smem_desc_sw128(smem_u32(sQ) + (kk - kMlaQTmemSteps) * 32, 16, 1024);
+              mma_bf16_ss(tS(js), qd, bd, idesc_s, 1u);
             }
-            mma_commit(smem_u32(&sfull[js % kMlaSBufs]));
-            ++js;
-            progressed = true;
           }
-          if (jp < js && mbar_test_wait(smem_u32(&pfull[jp % kMlaSBufs]), (jp / kMlaSBufs) & 1)) {
-            tc_fence_after();
-            const uint32_t va = smem_u32(sKV + (jp % kMlaStages) * kMlaStageBytes);
+          mma_commit(smem_u32(&sfull[js % kMlaSBufs]));
+        };
+        auto issue_pv = [&](int jp) {  // O += P_jp . V_jp, then release the stage
+          tc_fence_after();
+          const uint32_t va = smem_u32(sKV + (jp % kMlaStages) * kMlaStageBytes);
 #pragma unroll
-            for (int kk = 0; kk < kMlaBlk / 16; ++kk) {
-              const uint64_t bd = smem_desc_sw128(va + kk * 2048, kMlaKChunk, 1024);
-              mma_bf16_ts(tO, tS(jp) + kk * 8, bd, idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(smem_u32(&kvempty[jp % kMlaStages]));
-            ++jp;
-            progressed = true;
+          for (int kk = 0; kk < kMlaBlk / 16; ++kk) {
+            const uint64_t bd = smem_desc_sw128(va + kk * 2048, kMlaKChunk, 1024);
+            mma_bf16_ts(tO, tS(jp) + kk * 8, bd, idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
           }
-          if (progressed) {
-            t_last = globaltimer_ns();
-          } else if ((++spins & 63) == 0 && globaltimer_ns() - t_last > TO) {
-            report_error(kErrTimeout);  // neither input became ready in time
-            *abort_flag = 1;
+          mma_commit(smem_u32(&kvempty[jp % kMlaStages]));
+        };
+        // Fixed issue order S_0, S_1, S_2, then P_j.V followed by S_{j+3} (whose
+        // score buffer P_j.V frees). The softmax sends block j+1 ahead before it
+        // writes P_j, so S_{j+1} is always issued before the wait for P_j. Every
+        // wait suspends (try_wait), leaving issue slots to the softmax warps.
+        bool go = true;
+        for (int js = 0; go && js < kMlaSBufs && js < nblk; ++js) {
+          go = mbar_wait(smem_u32(&kvfull[js % kMlaStages]), (js / kMlaStages) & 1, TO, abort_flag);
+          if (go) issue_s(js);
+        }
+        for (int jp = 0; go && jp < nblk; ++jp) {
+          go = mbar_wait(smem_u32(&pfull[jp % kMlaSBufs]), (jp / kMlaSBufs) & 1, TO, abort_flag);
+          if (!go) break;
+          issue_pv(jp);
+          const int js = jp + kMlaSBufs;
+          if (js < nblk) {
+            go = mbar_wait(smem_u32(&kvfull[js % kMlaStages]), (js / kMlaStages) & 1, TO,
+                           abort_flag);
+            if (go) issue_s(js);
           }
         }
       }
@@ -331,21 +357,30 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t x_peer = mapa_shared(smem_u32(sX), peer);
     const uint32_t xfull_peer0 = mapa_shared(smem_u32(&xfull[0]), peer);
+    const uint32_t xfree_peer0 = mapa_shared(smem_u32(&xfree[0]), peer);
     const uint32_t xrow_off = (uint32_t)h * (kMlaXRow * 4) + (uint32_t)k0 * 4;
-    const bool announcer = (hf == 0 && h == 0);  // arms this CTA's xfull phases
+    const bool announcer = (hf == 0 && h == 0);  // re-arms xfull and returns credits
 
-    // Q slice -> TMEM (row h = lane h, two bf16 per column): column c holds
-    // dims d0 + 2c (c < 128) or r0 + 2(c - 128); this half stores columns
-    // [72 hf, 72 hf + 72) in steps of 8 columns (16 dims, 32 bytes).
+    // Q slice, row h = head h. Dims [0, 224) of the slice -> TMEM lane h, two
+    // bf16 per column (column c holds dims d0 + 2c, d0 + 2c + 1); this half
+    // stores columns [56 hf, 56 hf + 56) in steps of 8 columns (16 dims). The
+    // last 64 dims -> row h of the swizzled shared-memory chunk: half 0 stores
+    // value dims [d0 + 224, d0 + 256), half 1 the rope dims [r0, r0 + 32),
+    // as four 16-B pieces each.
     {
       const __nv_bfloat16* qrow = p.q + (t * kMlaHeads + h) * kMlaDqk;
       for (int c = hf * (kMlaQCols / 2); c < (hf + 1) * (kMlaQCols / 2); c += 8) {
-        const int dim = c < 128 ? d0 + 2 * c : r0 + 2 * (c - 128);
-        const uint4* src = reinterpret_cast<const uint4*>(qrow + dim);
+        const uint4* src = reinterpret_cast<const uint4*>(qrow + d0 + 2 * c);
         const uint4 x0 = __ldg(src), x1 = __ldg(src + 1);
         const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
         tmem_st8(tQ + c + lane_off, w);
       }
+      const uint4* src = reinterpret_cast<const uint4*>(qrow + (hf == 0 ? d0 + 224 : r0));
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint4*>(sQ + sw128_offset((uint32_t)h, (uint32_t)(4 * hf + i))) =
+            __ldg(src + i);
+      fence_proxy_async_smem();  // generic-proxy stores -> tensor-core reads
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(qfull));
@@ -366,20 +401,29 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     };
 
     float m_used = -INFINITY, l = 0.f;
-    float cur[kMlaHalf];
+    float cur[kMlaHalf], nxt[kMlaHalf];
     bool ok = true;
+    // Block j's own partial scores, from TMEM to the peer's exchange buffer
+    // j % 2. From block 2 on, that buffer is free once the peer has consumed
+    // block j-2 from it and handed back the credit.
+    auto load_and_send = [&](int j, float* v) {
+      bool r = warp_wait(smem_u32(&sfull[j % kMlaSBufs]), (j / kMlaSBufs) & 1, TO, abort_flag);
+      if (r && j >= kMlaXBufs)
+        r = warp_wait<true>(smem_u32(&xfree[j % kMlaXBufs]), ((j / kMlaXBufs) - 1) & 1, TO,
+                            abort_flag);
+      if (r) {
+        tc_fence_after();
+        load_s(j, v);
+        send(j, v);
+      }
+      return r;
+    };
+    if (nblk > 0) ok = load_and_send(0, cur);
     for (int j = 0; j < nblk; ++j) {
       const int xb = j % kMlaXBufs;
-      // (A) block j: own partial scores from TMEM, sent to the peer. The exchange
-      // buffer was last used for block j-3, which both CTAs consumed before
-      // sending blocks j-2 and j-1 that the other has waited on since.
-      if (announcer) mbar_arrive_expect_tx(smem_u32(&xfull[xb]), kMlaXPayload);
-      if (ok) ok = warp_wait(smem_u32(&sfull[j % kMlaSBufs]), (j / kMlaSBufs) & 1, TO, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        load_s(j, cur);
-        send(j, cur);
-      }
+      // (A) send ahead: block j+1 leaves before block j's softmax, so the
+      // exchange stays busy while this CTA waits for the peer's block j
+      if (ok && j + 1 < nblk) ok = load_and_send(j + 1, nxt);
       // (B) full scores = own partial + the peer's
       float mhalf = -INFINITY;
       if (ok) ok = warp_wait<true>(smem_u32(&xfull[xb]), (j / kMlaXBufs) & 1, TO, abort_flag);
@@ -410,6 +454,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       tc_fence_before();
       if (!named_barrier_and(2, 256, ok)) break;
       tc_fence_after();
+      // every thread has read exchange buffer xb (the values are consumed):
+      // arm it for block j+2 and hand the peer the credit to send that block.
+      // The credit is a relaxed arrival: a releasing one would first wait for
+      // this thread's own block j+1 stores to the peer to complete.
+      if (announcer && j + kMlaXBufs < nblk) {
+        mbar_arrive_expect_tx(smem_u32(&xfull[xb]), kMlaXPayload);
+        mbar_arrive_remote_relaxed(xfree_peer0 + (uint32_t)xb * 8u);
+      }
       const float mblk =
           fmaxf(sRed[((j & 1) * 2) * kMlaHeads + h], sRed[((j & 1) * 2 + 1) * kMlaHeads + h]);
       // lazy rescale: move the reference max only when it grows by more than 8 (x256)
@@ -457,6 +509,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         tc_fence_before();
         mbar_arrive(smem_u32(&pfull[j % kMlaSBufs]));
       }
+#pragma unroll
+      for (int i = 0; i < kMlaHalf; ++i) cur[i] = nxt[i];
     }
     // epilogue: every P.V product has finished once the last one has (in order)
     if (ok && nblk > 0)
