@@ -54,10 +54,14 @@ SCORE_BUDGET = 2 << 30  # bytes of fp32 score rows per chunk (as the library's o
 # ----------------------------------------------------------------------------------------
 # workload and algorithmic work
 # ----------------------------------------------------------------------------------------
-def make_problem(name: str, device, seed_offset: int = 0) -> synth.Problem:
+def make_problem(name: str, device, seed_offset: int = 0, batch=None) -> synth.Problem:
     w = dict(WORKLOADS[name])
     kind = w.pop("kind")
     w["seed"] = w["seed"] + 1000 * seed_offset
+    if batch is not None:  # smaller decode batches for profiler captures
+        if "batch" not in w:
+            raise SystemExit(f"--batch applies to decode workloads, not {name}")
+        w["batch"] = batch
     if kind == "paged":
         return synth.paged_decode(device=device, **w)
     if kind == "decode":
@@ -443,6 +447,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the decode batch (small cases for profiler captures)")
     ap.add_argument("--soak-s", type=float, default=1.0,
                     help="untimed seconds of steps right before the timed region (clock samples)")
     args = ap.parse_args(argv)
@@ -452,7 +458,7 @@ def main(argv=None):
         return reference_arm(args)
 
     world, rank, local = dist_setup(args.gpus)
-    p = make_problem(args.workload, "cuda", seed_offset=rank)
+    p = make_problem(args.workload, "cuda", seed_offset=rank, batch=args.batch)
     r = Runner(p)
     work = algorithmic_work(p)
     peaks = load_peaks()
@@ -502,7 +508,8 @@ def main(argv=None):
         cpu = cpu_baseline(p, args.workload)
 
     if rank == 0:
-        cfg = {"workload": args.workload, **WORKLOADS[args.workload], "k": K_SEL,
+        cfg = {"workload": args.workload, **WORKLOADS[args.workload],
+               **({"batch": args.batch} if args.batch else {}), "k": K_SEL,
                "heads": 128, "d_qk": 576, "d_v": 512, "h_idx": 64, "d_idx": 128,
                "query_rows_per_gpu": p.num_q,
                "l2": "inputs larger than L2 (no flush)",

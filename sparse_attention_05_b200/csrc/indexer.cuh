@@ -25,8 +25,9 @@
 //   warp 1      TMEM allocation + single-thread tcgen05.mma issue
 //   warps 2-3   query quantizers: bf16 -> E4M3 rows in the canonical swizzled
 //               K-major layout, w*s_q per row (double-buffered per unit)
-//   warps 4-11  epilogue: two warpgroups, each owning one of the two TMEM
-//               accumulators (tiles alternate between them); thread = key lane
+//   warps 4-11  epilogue: two warpgroups; tiles alternate between them and
+//               cycle through 512 / N TMEM accumulators (2 to 8), so the MMA
+//               can run that many tiles ahead; thread = key lane
 // A stage of the ring is reused only after the MMA has read its keys and the
 // epilogue has read its scales.
 #pragma once
@@ -47,7 +48,8 @@ constexpr int kIdxQBufBytes = 4 * kIdxHeads * kIdxDim;  // G <= 4 rows x 64 head
 constexpr int kIdxSmemBytes =
     1024 /*align slack*/ + kIdxStages * kIdxStageBytes + 2 * kIdxQBufBytes +
     2 * 4 * kIdxHeads * 4 /*wq*/ + kIdxStages * kIdxTile * 4 /*key scales*/ +
-    256 /*barriers etc*/ + 512 /*share + scan scratch*/;
+    512 /*barriers etc*/ + 512 /*share + scan scratch*/;
+constexpr int kIdxMaxAcc = 8;  // TMEM accumulators: 512 / N, at most 8
 
 struct IndexerParams {
   const __nv_bfloat16* q_idx;  // [T][64][128]
@@ -63,6 +65,7 @@ struct IndexerParams {
   int32_t G;                     // query rows per MMA (N = 64 G)
   int32_t groups_per_seq;        // ceil(row_count / G)
   int32_t num_groups;            // batch * groups_per_seq
+  int32_t scale_bulk;            // k_scale rows keep 16-B alignment for 4-key pieces
   uint64_t timeout_ns;
 };
 
@@ -181,18 +184,6 @@ __device__ void idx_share(const IndexerParams& p, IdxShare* out, uint32_t* scrat
   __syncthreads();
 }
 
-// Cache row of logical token s of sequence b (s must be < seqlen for paged).
-__device__ __forceinline__ int64_t idx_cache_row(const IndexerParams& p, int b, int s, bool& ok) {
-  ok = true;
-  if (!p.paged) return (int64_t)b * p.max_ctx + s;
-  const int page = __ldg(p.block_table + (int64_t)b * p.max_pages + s / p.page_size);
-  if (page < 0 || page >= p.num_pages) {
-    ok = false;
-    return 0;
-  }
-  return (int64_t)page * p.page_size + s % p.page_size;
-}
-
 __global__ void __launch_bounds__(kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ IndexerParams p,
                    const __grid_constant__ CUtensorMap tm_keys) {
@@ -207,8 +198,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + kIdxStages;
   uint64_t* tfull = bars + 2 * kIdxStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* qfull = tempty + 2;
+  uint64_t* tempty = tfull + kIdxMaxAcc;
+  uint64_t* qfull = tempty + kIdxMaxAcc;
   uint64_t* qempty = qfull + 2;
   uint64_t* mdone = qempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
@@ -218,16 +209,22 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = kIdxHeads * p.G;
-  const uint32_t tmem_cols = N * 2 <= 128 ? 128 : (N * 2 <= 256 ? 256 : 512);
+  // As many accumulators as tensor memory holds (an even number, so a given
+  // accumulator always belongs to the same epilogue warpgroup): the MMA runs
+  // up to nacc tiles ahead of the epilogue.
+  const int nacc = min(kIdxMaxAcc, 512 / N) & ~1;
+  const uint32_t tmem_cols = 512;
 
   if (tid == 0) {
     for (int s = 0; s < kIdxStages; ++s) {
       mbar_init(smem_u32(&kfull[s]), 1 + 32);    // expect_tx arrival + 32 scale copiers
       mbar_init(smem_u32(&kempty[s]), 1 + 128);  // MMA commit + the epilogue warpgroup
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kIdxMaxAcc; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);
       mbar_init(smem_u32(&tempty[i]), 128);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&qfull[i]), 64);
       mbar_init(smem_u32(&qempty[i]), 1 + 256);
     }
@@ -258,7 +255,22 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     while (!*abort_flag && idx_next(p, sh, cur, U)) {
       const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
       bool ok = true;
+      // Paged caches: lane l holds the page of half (l & 1) of tile kb + l / 2
+      // for a batch of 16 tiles starting at kb, and the next batch is already
+      // in flight, so no tile waits on a block-table load.
+      auto fetch_pages = [&](int kb) -> int {
+        const int kt = kb + (lane >> 1), s0 = kt * kIdxTile + (lane & 1) * 64;
+        if (!p.paged || kt >= U.kt1 || s0 > pos_max) return -1;
+        return __ldg(p.block_table + (int64_t)U.b * p.max_pages + s0 / p.page_size);
+      };
+      int kb = U.kt0;
+      int pg_cur = fetch_pages(kb), pg_nxt = fetch_pages(kb + 16);
       for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
+        if (kt - kb == 16) {
+          kb = kt;
+          pg_cur = pg_nxt;
+          pg_nxt = fetch_pages(kb + 16);
+        }
         const int st = it % kIdxStages;
         if (!warp_wait(smem_u32(&kempty[st]), ((it / kIdxStages) & 1) ^ 1, TO, abort_flag)) {
           ok = false;
@@ -271,11 +283,17 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int s0 = kt * kIdxTile + h * 64;
+          const int page = __shfl_sync(0xffffffffu, pg_cur, 2 * (kt - kb) + h);
           if (s0 <= pos_max) {
-            bool rok;
-            base[h] = idx_cache_row(p, U.b, s0, rok);
-            live[h] = rok;
-            if (!rok && lane == 0) report_error(kErrBounds);
+            if (!p.paged) {
+              base[h] = (int64_t)U.b * p.max_ctx + s0;
+              live[h] = true;
+            } else if (page >= 0 && page < p.num_pages) {
+              base[h] = (int64_t)page * p.page_size + s0 % p.page_size;
+              live[h] = true;
+            } else if (lane == 0) {
+              report_error(kErrBounds);
+            }
           }
         }
         if (lane == 0) {
@@ -285,14 +303,21 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             tma_load_2d(smem_u32(stages + st * kIdxStageBytes + h * 8192), &tm_keys, bar, 0,
                         (int)base[h]);
         }
-        // key scales: lane copies keys 4*lane .. 4*lane+3 of the tile
+        // key scales: lane l copies keys 4l .. 4l+3 of the tile, as one 16-B
+        // piece (zero-filled past the last visible key) when the cache rows
+        // keep 16-B alignment, else as four 4-B pieces
+        {
+          const int h = lane >> 4, e = lane * 4;
+          const int nvis = live[h] ? min(4, max(0, pos_max + 1 - (kt * kIdxTile + e))) : 0;
+          const float* src = p.k_scale + (nvis > 0 ? base[h] + (e & 63) : 0);
+          if (p.scale_bulk) {
+            cp_async_16(smem_u32(sscale + st * kIdxTile + e), src, 4u * (uint32_t)nvis);
+          } else {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int e = lane * 4 + v, h = e >> 6;
-          const int s = kt * kIdxTile + e;
-          const bool in = live[h] && s <= pos_max;
-          const float* src = p.k_scale + (in ? base[h] + (e & 63) : 0);
-          cp_async_4(smem_u32(sscale + st * kIdxTile + e), src, in ? 4u : 0u);
+            for (int v = 0; v < 4; ++v)
+              cp_async_4(smem_u32(sscale + st * kIdxTile + e + v), src + (v < nvis ? v : 0),
+                         v < nvis ? 4u : 0u);
+          }
         }
         cp_async_mbar_arrive(bar);
       }
@@ -317,9 +342,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         const uint32_t qaddr = smem_u32(qbuf + qb * kIdxQBufBytes);
         bool ok = true;
         for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
-          const int st = it % kIdxStages, ab = it & 1;
+          const int st = it % kIdxStages, ab = it % nacc;
           if (!mbar_wait(smem_u32(&kfull[st]), (it / kIdxStages) & 1, TO, abort_flag) ||
-              !mbar_wait(smem_u32(&tempty[ab]), ((it >> 1) & 1) ^ 1, TO, abort_flag)) {
+              !mbar_wait(smem_u32(&tempty[ab]), ((it / nacc) & 1) ^ 1, TO, abort_flag)) {
             ok = false;
             break;
           }
@@ -434,7 +459,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
         const float ks = sscale[st * kIdxTile + e];
         mbar_arrive(smem_u32(&kempty[st]));
-        if (!warp_wait(smem_u32(&tfull[wg]), (it >> 1) & 1, TO, abort_flag)) {
+        const int ab = (int)(it % (uint32_t)nacc);  // accumulator of this tile
+        if (!warp_wait(smem_u32(&tfull[ab]), (it / nacc) & 1, TO, abort_flag)) {
           ok = false;
           break;
         }
@@ -444,7 +470,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           // partial sums keep the FMA chains short
           float v0[32], v1[32];
           const uint32_t tcol =
-              tmem_base + ((uint32_t)(quad * 32) << 16) + wg * N + gi * kIdxHeads;
+              tmem_base + ((uint32_t)(quad * 32) << 16) + ab * N + gi * kIdxHeads;
           tmem_ld32(tcol, v0);
           tmem_ld32(tcol + 32, v1);
           tmem_wait_ld();
@@ -468,7 +494,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           p.scores[orow * p.ld + s] = out;
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&tempty[wg]));
+        mbar_arrive(smem_u32(&tempty[ab]));
       }
       if (!ok) break;
       mbar_arrive(smem_u32(&qempty[qb]));
