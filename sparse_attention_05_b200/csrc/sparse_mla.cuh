@@ -82,8 +82,10 @@ constexpr int kMlaResolve = 4 * kMlaBlk;      // keys the resolver handles per s
 constexpr int kMlaMaxSteps = (kMlaMaxK + kMlaResolve - 1) / kMlaResolve;  // 11
 constexpr int kMlaRowCap = kMlaMaxSteps * kMlaResolve;                   // 2112
 constexpr int kMlaMaskWords = kMlaRowCap / 32 + 2;
-constexpr int kMlaXRow = 52;                  // floats per exchange row (48 + pad)
-constexpr int kMlaXBytes = kMlaHeads * kMlaXRow * 4;
+// Exchange buffer: [12 four-key chunks][128 heads][4 floats], so that a warp's
+// 32 heads write (and read) 512 contiguous bytes per instruction.
+constexpr int kMlaXChunk = kMlaHeads * 16;    // bytes of one four-key chunk
+constexpr int kMlaXBytes = (kMlaBlk / 4) * kMlaXChunk;
 constexpr int kMlaXPayload = kMlaHeads * kMlaBlk * 4;  // bytes the peer sends per block
 constexpr int kMlaSmemBytes = 1024 + kMlaStages * kMlaStageBytes + kMlaQSmemBytes +
                               kMlaXBufs * kMlaXBytes + kMlaRowCap * 4 /*rows*/ +
@@ -119,7 +121,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* sKV = smem;
   uint8_t* sQ = sKV + kMlaStages * kMlaStageBytes;                      // [128][128 B] swizzled
-  uint8_t* sX = sQ + kMlaQSmemBytes;                                    // [2][128][52] f32
+  uint8_t* sX = sQ + kMlaQSmemBytes;                                    // [2][12][128][4] f32
   int32_t* sRow = reinterpret_cast<int32_t*>(sX + kMlaXBufs * kMlaXBytes);   // [2112]
   uint32_t* sBits = reinterpret_cast<uint32_t*>(sRow + kMlaRowCap);   // valid-key bits
   float* sRed = reinterpret_cast<float*>(sBits + kMlaMaskWords);      // [2][2][128]
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const uint32_t x_peer = mapa_shared(smem_u32(sX), peer);
     const uint32_t xfull_peer0 = mapa_shared(smem_u32(&xfull[0]), peer);
     const uint32_t xfree_peer0 = mapa_shared(smem_u32(&xfree[0]), peer);
-    const uint32_t xrow_off = (uint32_t)h * (kMlaXRow * 4) + (uint32_t)k0 * 4;
+    const uint32_t xrow_off = (uint32_t)(k0 / 4) * kMlaXChunk + (uint32_t)h * 16;
     const bool announcer = (hf == 0 && h == 0);  // re-arms xfull and returns credits
 
     // Q slice, row h = head h. Dims [0, 224) of the slice -> TMEM lane h, two
@@ -397,7 +399,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       const uint32_t bar = xfull_peer0 + xb * 8;
 #pragma unroll
       for (int c = 0; c < kMlaHalf / 4; ++c)
-        st_async_v4(dst + c * 16, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], bar);
+        st_async_v4(dst + c * kMlaXChunk, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], bar);
     };
 
     float m_used = -INFINITY, l = 0.f;
@@ -428,10 +430,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       float mhalf = -INFINITY;
       if (ok) ok = warp_wait<true>(smem_u32(&xfull[xb]), (j / kMlaXBufs) & 1, TO, abort_flag);
       if (ok) {
-        const float* xr = reinterpret_cast<const float*>(sX + xb * kMlaXBytes + xrow_off);
+        const uint8_t* xr = sX + xb * kMlaXBytes + xrow_off;
 #pragma unroll
         for (int c = 0; c < kMlaHalf / 4; ++c) {
-          const float4 v = reinterpret_cast<const float4*>(xr)[c];
+          const float4 v = *reinterpret_cast<const float4*>(xr + c * kMlaXChunk);
           cur[4 * c] += v.x;
           cur[4 * c + 1] += v.y;
           cur[4 * c + 2] += v.z;
