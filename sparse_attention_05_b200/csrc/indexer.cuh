@@ -465,29 +465,33 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           break;
         }
         tc_fence_after();
+        // Row gi's 64 head columns come as two 32-column chunks (A: heads
+        // 0-31, B: heads 32-63). The next chunk's load is always in flight
+        // while the current one is reduced, so the tensor-memory load latency
+        // hides behind the ReLU / weighted head sum.
+        const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * N;
+        uint32_t ca[32], cb[32];
+        tmem_ld32u(tcol, ca);
+        tmem_wait_ld_fence(ca);
         for (int gi = 0; gi < U.nrows; ++gi) {
-          // both 32-column loads in flight before one wait; four independent
-          // partial sums keep the FMA chains short
-          float v0[32], v1[32];
-          const uint32_t tcol =
-              tmem_base + ((uint32_t)(quad * 32) << 16) + ab * N + gi * kIdxHeads;
-          tmem_ld32(tcol, v0);
-          tmem_ld32(tcol + 32, v1);
-          tmem_wait_ld();
           const float4* w4 = reinterpret_cast<const float4*>(wrow + gi * kIdxHeads);
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          auto reduce32 = [&](const uint32_t (&v)[32], const float4* wq4) {
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 wa = w4[q4], wb = w4[8 + q4];
-            a0 = fmaf(wa.x, fmaxf(v0[4 * q4 + 0], 0.f), a0);
-            a1 = fmaf(wa.y, fmaxf(v0[4 * q4 + 1], 0.f), a1);
-            a2 = fmaf(wa.z, fmaxf(v0[4 * q4 + 2], 0.f), a2);
-            a3 = fmaf(wa.w, fmaxf(v0[4 * q4 + 3], 0.f), a3);
-            a0 = fmaf(wb.x, fmaxf(v1[4 * q4 + 0], 0.f), a0);
-            a1 = fmaf(wb.y, fmaxf(v1[4 * q4 + 1], 0.f), a1);
-            a2 = fmaf(wb.z, fmaxf(v1[4 * q4 + 2], 0.f), a2);
-            a3 = fmaf(wb.w, fmaxf(v1[4 * q4 + 3], 0.f), a3);
-          }
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const float4 wv = wq4[q4];
+              a0 = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * q4 + 0]), 0.f), a0);
+              a1 = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * q4 + 1]), 0.f), a1);
+              a2 = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * q4 + 2]), 0.f), a2);
+              a3 = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * q4 + 3]), 0.f), a3);
+            }
+          };
+          tmem_ld32u(tcol + gi * kIdxHeads + 32, cb);
+          reduce32(ca, w4);
+          tmem_wait_ld_fence(cb);
+          if (gi + 1 < U.nrows) tmem_ld32u(tcol + (gi + 1) * kIdxHeads, ca);
+          reduce32(cb, w4 + 8);
+          if (gi + 1 < U.nrows) tmem_wait_ld_fence(ca);
           const float acc = (a0 + a1) + (a2 + a3);
           const float out = (s <= pos0 + gi) ? ks * acc : -INFINITY;
           const int64_t orow = (int64_t)U.b * p.row_count + (U.i0 - p.row_begin) + gi;
