@@ -216,31 +216,47 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
     r = min(r, (uint32_t)kTopkSample);
     uint32_t tau_low, unused;
     find_kth(kTopkSample, r, [&](int e, int) { return sample[e]; }, hist, misc, tau_low, unused);
-    // keep keys >= tau_low in position order (4 consecutive keys per thread)
+    // keep keys >= tau_low in position order: 16 consecutive keys per thread
+    // per step, with the next step's four 16-B loads already in flight
+    constexpr int kStep = 16 * kTopkThreads;
+    auto load16 = [&](int base, float4 (&v)[4]) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e0 = base + 16 * tid + 4 * u;
+        if (e0 + 3 < n) {  // rows start 16-B aligned (ld is a multiple of 4)
+          v[u] = *reinterpret_cast<const float4*>(row + e0);
+        } else {
+          v[u].x = e0 < n ? row[e0] : -INFINITY;
+          v[u].y = e0 + 1 < n ? row[e0 + 1] : -INFINITY;
+          v[u].z = e0 + 2 < n ? row[e0 + 2] : -INFINITY;
+          v[u].w = e0 + 3 < n ? row[e0 + 3] : -INFINITY;
+        }
+      }
+    };
     uint32_t m_run = 0;
     bool overflow = false;
+    float4 cur4[4], nxt4[4];
+    load16(0, cur4);
 #pragma unroll 1
-    for (int base = 0; base < n; base += 4 * kTopkThreads) {
-      const int e0 = base + 4 * tid;
-      uint32_t kk[4];
-      uint32_t c = 0;
-      if (e0 + 3 < n) {  // rows start 16-B aligned (ld is a multiple of 4)
-        const float4 v = *reinterpret_cast<const float4*>(row + e0);
-        kk[0] = score_key(v.x);
-        kk[1] = score_key(v.y);
-        kk[2] = score_key(v.z);
-        kk[3] = score_key(v.w);
-      } else {
+    for (int base = 0; base < n; base += kStep) {
+      if (base + kStep < n) load16(base + kStep, nxt4);
+      uint32_t kk[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) kk[u] = (e0 + u < n) ? score_key(row[e0 + u]) : 0u;
+      for (int u = 0; u < 4; ++u) {
+        kk[4 * u] = score_key(cur4[u].x);
+        kk[4 * u + 1] = score_key(cur4[u].y);
+        kk[4 * u + 2] = score_key(cur4[u].z);
+        kk[4 * u + 3] = score_key(cur4[u].w);
       }
+      const int e0 = base + 16 * tid;
+      uint32_t c = 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) c += (e0 + u < n) && kk[u] >= tau_low;
+      for (int u = 0; u < 16; ++u) c += (e0 + u < n) && kk[u] >= tau_low;
       const uint32_t excl = block_exclusive_scan(c, misc, misc + 32);
       const uint32_t tot = misc[32];
       uint32_t w = m_run + excl;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 16; ++u) {
         if ((e0 + u < n) && kk[u] >= tau_low) {
           if (w < (uint32_t)kTopkCandCap) {
             cand_key[w] = kk[u];
@@ -253,6 +269,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
       overflow = m_run > (uint32_t)kTopkCandCap;
       __syncthreads();
       if (overflow) break;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) cur4[u] = nxt4[u];
     }
     if (!overflow && m_run >= k) {
       const int m = (int)m_run;
@@ -269,20 +287,33 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
     return;
   }
 
-  // ---- short rows: cached in shared memory across the passes ---------------------
-  // (n <= 4k <= 8192 <= kTopkCacheElems)
-  find_kth(n, k,
-           [&](int e, int pass) {
-             float x;
-             if (pass == 0) {
-               x = row[e];
-               cache[e] = x;
-             } else {
-               x = cache[e];
-             }
-             return score_key(x);
-           },
-           hist, misc, tau, r_eq);
+  // ---- short rows: staged in shared memory (all loads in flight), then selected ----
+  // (n <= 4k <= 8192 <= kTopkCacheElems; rows start 16-B aligned)
+  {
+    constexpr int kPer = 4 * kTopkThreads;
+    float4 v[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int e0 = h * kPer + 4 * tid;
+      if (e0 + 3 < n) {
+        v[h] = *reinterpret_cast<const float4*>(row + e0);
+      } else {
+        v[h].x = e0 < n ? row[e0] : -INFINITY;
+        v[h].y = e0 + 1 < n ? row[e0 + 1] : -INFINITY;
+        v[h].z = e0 + 2 < n ? row[e0 + 2] : -INFINITY;
+        v[h].w = e0 + 3 < n ? row[e0 + 3] : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int e0 = h * kPer + 4 * tid;
+      if (e0 < n) *reinterpret_cast<float4*>(cache + e0) = v[h];
+    }
+    for (int e0 = 2 * kPer + 4 * tid; e0 < n; e0 += kPer)  // not reached for k <= 2048
+      for (int u = 0; u < 4 && e0 + u < n; ++u) cache[e0 + u] = row[e0 + u];
+    __syncthreads();
+  }
+  find_kth(n, k, [&](int e, int) { return score_key(cache[e]); }, hist, misc, tau, r_eq);
   compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(cache[e]); },
                [&](int e) { return e; }, out, misc);
 }

@@ -102,3 +102,64 @@ def test_host_argument_checks():
     assert e.value.status == 1
     with pytest.raises(dsa.DSAError):
         dsa.dsa_indexer_scores(p.q_idx, p.w, p.k_idx, p.k_scale, kv, 3)  # T != B * q_per_seq
+
+
+_BF16_POS = (np.arange(1, 0x7F80, dtype=np.uint32) << 16).view(np.float32)  # positive finite bf16
+
+
+def _midpoint_distance(x: np.ndarray, amax) -> np.ndarray:
+    """fp32 ulps between RN(x / s_q) (s_q = RN(amax / 448)) and the nearest
+    E4M3 rounding midpoint, for quotients in the normal E4M3 range."""
+    s_q = np.float32(amax) / np.float32(448.0)
+    quot = (x / s_q).astype(np.float32)
+    rem = (quot.view(np.uint32) & 0xFFFFF).astype(np.int64)
+    return np.where(quot >= np.float32(2.0 ** -6), np.abs(rem - 0x80000), 1 << 30)
+
+
+def _near_midpoint_row(rng) -> np.ndarray:
+    """128 bf16 values, the hardest inputs for the query quantization: amax is
+    chosen among bf16 values in [0.5, 8) so that many values below it have a
+    fp32 quotient RN(x / s_q) within a few ulps of an E4M3 rounding midpoint
+    (or exactly on one, where ties-to-even decides); the row is amax plus the
+    127 values closest to midpoints, with random signs, in random order."""
+    amaxes = _BF16_POS[(_BF16_POS >= 0.5) & (_BF16_POS < 8.0)]
+    best = []
+    for amax in rng.choice(amaxes, 48, replace=False):
+        d = _midpoint_distance(_BF16_POS[_BF16_POS < amax], amax)
+        best.append((int(d.min()), -int((d <= 16).sum()), float(amax)))
+    amax = np.float32(min(best)[2])
+    x = _BF16_POS[_BF16_POS < amax]
+    pick = x[np.argsort(_midpoint_distance(x, amax), kind="stable")[:127]]
+    row = np.concatenate([[amax], pick * rng.choice([-1.0, 1.0], 127)])
+    return rng.permutation(row).astype(np.float32)
+
+
+def test_query_codes_exact_via_one_hot_keys():
+    """Every E4M3 query code is checked exactly: keys are +-e_i (scale 1) and
+    each row weights one head by 1, so score(row, key +-e_i) = RN(s_q * ReLU(
+    +-q_hat_i)) on both sides; the GPU must equal the oracle bit for bit.
+    Half the rows hold values whose quotients sit next to E4M3 midpoints."""
+    B, H, D = 64, 64, 128
+    p = synth.decode(batch=B, ctx=2 * D, q_per_seq=1, seed=36)
+    rng = np.random.default_rng(36)
+    q = p.q_idx.float().numpy().copy()
+    for b in range(B):
+        if b % 2 == 0:
+            q[b, b % H] = _near_midpoint_row(rng)
+    p.q_idx = torch.from_numpy(q).to(torch.bfloat16)
+    assert torch.equal(p.q_idx.float(), torch.from_numpy(q))  # values are bf16-exact
+    w = np.zeros((B, H), np.float32)
+    w[np.arange(B), np.arange(B) % H] = 1.0
+    p.w = torch.from_numpy(w)
+    codes = np.zeros((B, 2 * D, D), np.uint8)
+    for i in range(D):
+        codes[:, i, i] = 0x38        # +1.0 in E4M3
+        codes[:, D + i, i] = 0xB8    # -1.0
+    p.k_idx = torch.from_numpy(codes)
+    p.k_scale = torch.ones(B, 2 * D)
+    got = _gpu_scores(p)
+    a = oracle_args(p)
+    ref = indexer_scores(a["q_idx"], a["w"], a["k_idx"], a["k_scale"], a["q_seq"], a["q_pos"],
+                         ld=got.shape[1], block_table=None)
+    bad = got[:, :2 * D] != ref[:, :2 * D]
+    assert not bad.any(), f"{bad.sum()} scores differ; first at {np.argwhere(bad)[0]}"
