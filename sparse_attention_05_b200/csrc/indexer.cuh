@@ -381,14 +381,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       uint8_t* qdst = qbuf + qb * kIdxQBufBytes;
       float* wdst = wq + qb * 4 * kIdxHeads;
       // A half-warp converts one 128-element row (8 elements = 16 B per lane);
-      // 8 rows per half-warp are loaded before any is used, so their global
-      // load latencies overlap. Rows r = base + 4 i of the batch.
+      // kQRows rows per half-warp are loaded before any is used, so their
+      // global load latencies overlap (the loads compete with every CTA's key
+      // stream, so each round trip is long). Rows r = base + 4 i of the batch.
+      constexpr int kQRows = 16;
       const int half = lane >> 4, hl = lane & 15;
-      for (int base = qw * 2 + half; base < N; base += 32) {
-        uint4 raw[8];
-        float wj[8];
+      for (int base = qw * 2 + half; base < N; base += 4 * kQRows) {
+        uint4 raw[kQRows];
+        float wj[kQRows];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kQRows; ++i) {
           const int r = base + 4 * i;
           const int gi = r / kIdxHeads, j = r % kIdxHeads;
           raw[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -401,8 +403,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = base + 4 * i;
+        for (int i = 0; i < kQRows; ++i) {
+          const int r = base + 4 * i;  // < N: N is a multiple of 64
           const uint32_t wv[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
           float x[8];
 #pragma unroll
