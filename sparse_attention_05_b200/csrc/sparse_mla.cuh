@@ -36,20 +36,25 @@
 //                          dims per copy, 128-B swizzle, zero fill for row -1),
 //                          warps 11-15 copy rows 24-47 in 16-B cp.async pieces
 //                          (zero fill for row -1) into the same swizzled
-//                          4-stage ring; both complete the stage barrier
+//                          5-stage ring; both complete the stage barrier
 //   MMA (warp 10)          S_j = Q . K_j^T (M=128 heads, N=48, K=288, Q from
 //                          TMEM) and O += P_j . V_j (M=128, N=256, K=48, P from
 //                          TMEM, V MN-major), each issued as soon as it is ready
-//   softmax (warps 2-9)    thread = (head, half of the block's keys). The
-//                          exchange is the scarcest resource (distributed shared
-//                          memory moves ~20 GB/s per SM), so it never idles:
-//                          block j+1's partial scores are sent to the peer
-//                          before block j's softmax runs. The peer's partials
-//                          land in a two-buffer ring; after consuming a buffer
-//                          this CTA re-arms it and hands the peer a credit (a
-//                          remote mbarrier arrival) for the block two ahead.
-//                          Online softmax in base 2 with a lazy rescale of O
-//                          (only when the running max grows by more than 8).
+//   softmax (warps 2-9)    thread = (head, half of the block's keys). Heads
+//                          have owners: CTA r runs the online softmax of heads
+//                          [64 r, 64 r + 64); its other 128 threads serve the
+//                          peer's heads, sending their partial scores one block
+//                          ahead and writing the P (bf16) and rescale factors
+//                          the peer sends back into their TMEM lanes. Per key
+//                          and direction 256 B of partial scores and 128 B of
+//                          P cross the cluster (not 512 B), and each CTA
+//                          exponentiates only 64 heads. Inboxes are two-buffer
+//                          rings laid out [16-B chunk][head] (every warp store
+//                          is 512 contiguous bytes), guarded by credits (relaxed
+//                          remote mbarrier arrivals). Online softmax in base 2
+//                          with a lazy rescale of O (only when the running max
+//                          grows by more than 8), which the owner's factor
+//                          carries to the peer's half of O.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -63,7 +68,7 @@ constexpr int kMlaDqk = 576;
 constexpr int kMlaDv = 512;
 constexpr int kMlaBlk = 48;                   // keys per block
 constexpr int kMlaHalf = kMlaBlk / 2;         // keys per softmax thread
-constexpr int kMlaStages = 4;                 // gather ring
+constexpr int kMlaStages = 5;                 // gather ring
 constexpr int kMlaSBufs = 3;                  // TMEM score / probability buffers
 constexpr int kMlaXBufs = 2;                  // exchange ring (credit based)
 constexpr int kMlaThreads = 512;              // TMA, resolver, 8 softmax, MMA, 5 cp.async warps
@@ -82,13 +87,20 @@ constexpr int kMlaResolve = 4 * kMlaBlk;      // keys the resolver handles per s
 constexpr int kMlaMaxSteps = (kMlaMaxK + kMlaResolve - 1) / kMlaResolve;  // 11
 constexpr int kMlaRowCap = kMlaMaxSteps * kMlaResolve;                   // 2112
 constexpr int kMlaMaskWords = kMlaRowCap / 32 + 2;
-// Exchange buffer: [12 four-key chunks][128 heads][4 floats], so that a warp's
-// 32 heads write (and read) 512 contiguous bytes per instruction.
-constexpr int kMlaXChunk = kMlaHeads * 16;    // bytes of one four-key chunk
-constexpr int kMlaXBytes = (kMlaBlk / 4) * kMlaXChunk;
-constexpr int kMlaXPayload = kMlaHeads * kMlaBlk * 4;  // bytes the peer sends per block
+// Exchange inboxes, laid out [16-B chunk][64 heads of the owner] so that a
+// warp's 32 heads write (and read) 512 contiguous bytes per instruction:
+//   partial scores of this CTA's own heads from the peer: 12 chunks of 4 keys;
+//   P (bf16) of the peer's heads from the peer: 6 chunks of 8 keys, then one
+//   fp32 rescale factor per head.
+constexpr int kMlaXsChunk = 64 * 16;
+constexpr int kMlaXsBytes = (kMlaBlk / 4) * kMlaXsChunk;     // 12 KB
+constexpr int kMlaXsPayload = kMlaXsBytes;
+constexpr int kMlaXpFactor = (kMlaBlk / 8) * kMlaXsChunk;    // 6 KB of P
+constexpr int kMlaXpBytes = kMlaXpFactor + 64 * 4;
+constexpr int kMlaXpPayload = kMlaXpBytes;
 constexpr int kMlaSmemBytes = 1024 + kMlaStages * kMlaStageBytes + kMlaQSmemBytes +
-                              kMlaXBufs * kMlaXBytes + kMlaRowCap * 4 /*rows*/ +
+                              kMlaXBufs * (kMlaXsBytes + kMlaXpBytes) + 256 /*peer's sums*/ +
+                              2 * kMlaHeads * 4 /*own sums*/ + kMlaRowCap * 4 /*rows*/ +
                               kMlaMaskWords * 4 /*valid bits*/ + 2 * 2 * kMlaHeads * 4 /*max swap*/ +
                               40 * 8 /*barriers*/ + 16;
 static_assert(kMlaSmemBytes <= 232448, "sparse MLA shared memory exceeds the per-CTA limit");
@@ -121,8 +133,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* sKV = smem;
   uint8_t* sQ = sKV + kMlaStages * kMlaStageBytes;                      // [128][128 B] swizzled
-  uint8_t* sX = sQ + kMlaQSmemBytes;                                    // [2][12][128][4] f32
-  int32_t* sRow = reinterpret_cast<int32_t*>(sX + kMlaXBufs * kMlaXBytes);   // [2112]
+  uint8_t* sXs = sQ + kMlaQSmemBytes;                                   // [2] partial-score inbox
+  uint8_t* sXp = sXs + kMlaXBufs * kMlaXsBytes;                          // [2] P inbox
+  uint8_t* sLfin = sXp + kMlaXBufs * kMlaXpBytes;                        // [64] peer's sums
+  float* sLh = reinterpret_cast<float*>(sLfin + 256);                    // [2][128] own sums
+  int32_t* sRow = reinterpret_cast<int32_t*>(sLh + 2 * kMlaHeads);      // [2112]
   uint32_t* sBits = reinterpret_cast<uint32_t*>(sRow + kMlaRowCap);   // valid-key bits
   float* sRed = reinterpret_cast<float*>(sBits + kMlaMaskWords);      // [2][2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRed + 2 * 2 * kMlaHeads);
@@ -130,9 +145,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   uint64_t* kvempty = kvfull + kMlaStages;      // [stages] O += P V of the stage's block done
   uint64_t* sfull = kvempty + kMlaStages;       // [2] S in score buffer
   uint64_t* pfull = sfull + kMlaSBufs;          // [2] P written over S
-  uint64_t* xfull = pfull + kMlaSBufs;          // [2] peer's partial scores arrived
-  uint64_t* xfree = xfull + kMlaXBufs;          // [2] the peer consumed this CTA's send (credit)
-  uint64_t* qfull = xfree + kMlaXBufs;          // Q stored in TMEM and shared memory
+  uint64_t* xsfull = pfull + kMlaSBufs;         // [2] peer's partial scores (own heads) arrived
+  uint64_t* xsfree = xsfull + kMlaXBufs;        // [2] credit: the peer consumed our partials
+  uint64_t* xpfull = xsfree + kMlaXBufs;        // [2] peer's P (its heads) arrived
+  uint64_t* xpfree = xpfull + kMlaXBufs;        // [2] credit: the peer consumed our P
+  uint64_t* lfull = xpfree + kMlaXBufs;         // the peer's softmax sums arrived
+  uint64_t* qfull = lfull + 1;                  // Q stored in TMEM and shared memory
   uint64_t* mdone = qfull + 1;
   uint64_t* rready = mdone + 1;                 // [11] resolver step done
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(rready + kMlaMaxSteps);
@@ -161,17 +179,23 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       mbar_init(smem_u32(&pfull[i]), 256);
     }
     for (int i = 0; i < kMlaXBufs; ++i) {
-      mbar_init(smem_u32(&xfull[i]), 1);  // + the peer's bytes
-      mbar_init(smem_u32(&xfree[i]), 1);  // one remote arrival from the peer
+      mbar_init(smem_u32(&xsfull[i]), 1);  // + the peer's bytes
+      mbar_init(smem_u32(&xsfree[i]), 1);  // one remote arrival from the peer
+      mbar_init(smem_u32(&xpfull[i]), 1);
+      mbar_init(smem_u32(&xpfree[i]), 1);
     }
+    mbar_init(smem_u32(lfull), 1);
     mbar_init(smem_u32(qfull), 256);
     mbar_init(smem_u32(mdone), 1);
     for (int i = 0; i < kMlaMaxSteps; ++i) mbar_init(smem_u32(&rready[i]), 1);
     *abort_flag = 0;
     // the first two blocks' exchange buffers start free: arm them before the
     // peer may send (later blocks are armed when their buffer is consumed)
-    for (int i = 0; i < kMlaXBufs && i < nblk; ++i)
-      mbar_arrive_expect_tx(smem_u32(&xfull[i]), kMlaXPayload);
+    for (int i = 0; i < kMlaXBufs && i < nblk; ++i) {
+      mbar_arrive_expect_tx(smem_u32(&xsfull[i]), kMlaXsPayload);
+      mbar_arrive_expect_tx(smem_u32(&xpfull[i]), kMlaXpPayload);
+    }
+    mbar_arrive_expect_tx(smem_u32(lfull), 64 * 4);
     fence_mbarrier_init_cluster();
   }
   if (warp == kMlaMmaWarp) {
@@ -352,16 +376,23 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax / epilogue
+    // Heads have owners: CTA r runs the online softmax of heads [64 r, 64 r + 64)
+    // (its TMEM lane quadrants 2r, 2r+1). Its other 128 threads serve the peer's
+    // heads: they send the peer those heads' partial scores (ahead, one block in
+    // flight) and receive the peer's P (bf16) and rescale factors back into
+    // their TMEM lanes. Per key and direction 256 B of partial scores and 128 B
+    // of P cross the cluster instead of 512 B, and each CTA exponentiates only
+    // its own 64 heads.
     const int quad = warp & 3;               // TMEM lane quadrant
     const int hf = (warp - 2) >> 2;          // which half of each block's keys
     const int h = quad * 32 + lane;          // head == TMEM lane
+    const int hl = h & 63;                   // head within its owner's 64
     const int k0 = hf * kMlaHalf;            // first key (column) of this half
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t x_peer = mapa_shared(smem_u32(sX), peer);
-    const uint32_t xfull_peer0 = mapa_shared(smem_u32(&xfull[0]), peer);
-    const uint32_t xfree_peer0 = mapa_shared(smem_u32(&xfree[0]), peer);
-    const uint32_t xrow_off = (uint32_t)(k0 / 4) * kMlaXChunk + (uint32_t)h * 16;
-    const bool announcer = (hf == 0 && h == 0);  // re-arms xfull and returns credits
+    const bool own = (h >> 6) == (int)rank;
+    const bool announcer = (hf == 0 && hl == 0);  // re-arms this group's inbox, returns credits
+    const uint32_t xs_off = (uint32_t)(hf * (kMlaHalf / 4)) * kMlaXsChunk + (uint32_t)hl * 16;
+    const uint32_t xp_off = (uint32_t)(hf * (kMlaHalf / 8)) * kMlaXsChunk + (uint32_t)hl * 16;
 
     // Q slice, row h = head h. Dims [0, 224) of the slice -> TMEM lane h, two
     // bf16 per column (column c holds dims d0 + 2c, d0 + 2c + 1); this half
@@ -393,106 +424,96 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       tmem_ld8(tS(j) + k0 + 16 + lane_off, v + 16);
       tmem_wait_ld();
     };
-    auto send = [&](int j, const float* v) {  // partial scores of block j -> peer
-      const uint32_t xb = (uint32_t)(j % kMlaXBufs);
-      const uint32_t dst = x_peer + xb * kMlaXBytes + xrow_off;
-      const uint32_t bar = xfull_peer0 + xb * 8;
+    // O rows of head h, this thread's 128 of the CTA's 256 value columns, x f
+    auto rescale_o = [&](float f) {
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        const uint32_t col = tO + hf * 128 + c * 32 + lane_off;
+        tmem_ld32(col, o);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < kMlaHalf / 4; ++c)
-        st_async_v4(dst + c * kMlaXChunk, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], bar);
+        for (int i = 0; i < 32; ++i) o[i] *= f;
+        tmem_st32(col, o);
+      }
+      tmem_wait_st();
+    };
+    auto write_p = [&](int j, const uint32_t* pk) {  // P_j over S_j, then release it to the MMA
+      tmem_st8(tS(j) + hf * (kMlaHalf / 2) + lane_off, pk);
+      tmem_st4(tS(j) + hf * (kMlaHalf / 2) + 8 + lane_off, pk + 8);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&pfull[j % kMlaSBufs]));
     };
 
     float m_used = -INFINITY, l = 0.f;
-    float cur[kMlaHalf], nxt[kMlaHalf];
     bool ok = true;
-    // Block j's own partial scores, from TMEM to the peer's exchange buffer
-    // j % 2. From block 2 on, that buffer is free once the peer has consumed
-    // block j-2 from it and handed back the credit.
-    auto load_and_send = [&](int j, float* v) {
-      bool r = warp_wait(smem_u32(&sfull[j % kMlaSBufs]), (j / kMlaSBufs) & 1, TO, abort_flag);
-      if (r && j >= kMlaXBufs)
-        r = warp_wait<true>(smem_u32(&xfree[j % kMlaXBufs]), ((j / kMlaXBufs) - 1) & 1, TO,
-                            abort_flag);
-      if (r) {
-        tc_fence_after();
-        load_s(j, v);
-        send(j, v);
-      }
-      return r;
-    };
-    if (nblk > 0) ok = load_and_send(0, cur);
-    for (int j = 0; j < nblk; ++j) {
-      const int xb = j % kMlaXBufs;
-      // (A) send ahead: block j+1 leaves before block j's softmax, so the
-      // exchange stays busy while this CTA waits for the peer's block j
-      if (ok && j + 1 < nblk) ok = load_and_send(j + 1, nxt);
-      // (B) full scores = own partial + the peer's
-      float mhalf = -INFINITY;
-      if (ok) ok = warp_wait<true>(smem_u32(&xfull[xb]), (j / kMlaXBufs) & 1, TO, abort_flag);
-      if (ok) {
-        const uint8_t* xr = sX + xb * kMlaXBytes + xrow_off;
-#pragma unroll
-        for (int c = 0; c < kMlaHalf / 4; ++c) {
-          const float4 v = *reinterpret_cast<const float4*>(xr + c * kMlaXChunk);
-          cur[4 * c] += v.x;
-          cur[4 * c + 1] += v.y;
-          cur[4 * c + 2] += v.z;
-          cur[4 * c + 3] += v.w;
-        }
-        ok = warp_wait(smem_u32(&kvfull[j % kMlaStages]), (j / kMlaStages) & 1, TO, abort_flag);
-      }
-      if (ok) {
-        const int b0 = j * kMlaBlk + k0;  // this half's 24 valid-key bits
-        const uint64_t w2 = ((uint64_t)sBits[(b0 >> 5) + 1] << 32) | sBits[b0 >> 5];
-        const uint32_t mask = (uint32_t)(w2 >> (b0 & 31)) & 0xFFFFFFu;
-#pragma unroll
-        for (int i = 0; i < kMlaHalf; ++i) {
-          cur[i] = ((mask >> i) & 1u) ? cur[i] * p.scale_log2 : -INFINITY;
-          mhalf = fmaxf(mhalf, cur[i]);
-        }
-        sRed[((j & 1) * 2 + hf) * kMlaHeads + h] = mhalf;
-      }
-      // both halves of a head agree on the block max (and on whether to go on)
-      tc_fence_before();
-      if (!named_barrier_and(2, 256, ok)) break;
-      tc_fence_after();
-      // every thread has read exchange buffer xb (the values are consumed):
-      // arm it for block j+2 and hand the peer the credit to send that block.
-      // The credit is a relaxed arrival: a releasing one would first wait for
-      // this thread's own block j+1 stores to the peer to complete.
-      if (announcer && j + kMlaXBufs < nblk) {
-        mbar_arrive_expect_tx(smem_u32(&xfull[xb]), kMlaXPayload);
-        mbar_arrive_remote_relaxed(xfree_peer0 + (uint32_t)xb * 8u);
-      }
-      const float mblk =
-          fmaxf(sRed[((j & 1) * 2) * kMlaHeads + h], sRed[((j & 1) * 2 + 1) * kMlaHeads + h]);
-      // lazy rescale: move the reference max only when it grows by more than 8 (x256)
-      const bool grow = mblk > m_used + 8.0f;
-      const bool need_o = grow && m_used != -INFINITY;  // O already holds earlier blocks
-      if (__any_sync(0xffffffffu, need_o)) {
-        // O += P_{j-1} V_{j-1} must have finished before O is touched
-        if (!warp_wait(smem_u32(&kvempty[(j - 1) % kMlaStages]), ((j - 1) / kMlaStages) & 1, TO,
-                       abort_flag)) {
-          ok = false;
-        } else {
+    if (own) {
+      // ---------------------------------------------------- owner of heads h
+      const uint32_t xp_peer = mapa_shared(smem_u32(sXp), peer);
+      const uint32_t xpfull_peer0 = mapa_shared(smem_u32(&xpfull[0]), peer);
+      const uint32_t xsfree_peer0 = mapa_shared(smem_u32(&xsfree[0]), peer);
+      float cur[kMlaHalf];
+      for (int j = 0; j < nblk; ++j) {
+        const int xb = j % kMlaXBufs;
+        float mhalf = -INFINITY;
+        if (ok) ok = warp_wait(smem_u32(&sfull[j % kMlaSBufs]), (j / kMlaSBufs) & 1, TO, abort_flag);
+        if (ok) {
           tc_fence_after();
-          const float f = need_o ? ex2_approx(m_used - mblk) : 1.0f;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {  // this half's 128 columns of O
-            float o[32];
-            const uint32_t col = tO + hf * 128 + c * 32 + lane_off;
-            tmem_ld32(col, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= f;
-            tmem_st32(col, o);
-          }
-          tmem_wait_st();
-          l *= f;
+          load_s(j, cur);
+          ok = warp_wait<true>(smem_u32(&xsfull[xb]), (j / kMlaXBufs) & 1, TO, abort_flag);
         }
-      }
-      if (grow) m_used = mblk;
-      if (ok) {
+        if (ok) {  // full scores = own partial + the peer's
+          const uint8_t* xr = sXs + xb * kMlaXsBytes + xs_off;
+#pragma unroll
+          for (int c = 0; c < kMlaHalf / 4; ++c) {
+            const float4 v = *reinterpret_cast<const float4*>(xr + c * kMlaXsChunk);
+            cur[4 * c] += v.x;
+            cur[4 * c + 1] += v.y;
+            cur[4 * c + 2] += v.z;
+            cur[4 * c + 3] += v.w;
+          }
+          ok = warp_wait(smem_u32(&kvfull[j % kMlaStages]), (j / kMlaStages) & 1, TO, abort_flag);
+        }
+        if (ok) {
+          const int b0 = j * kMlaBlk + k0;  // this half's 24 valid-key bits
+          const uint64_t w2 = ((uint64_t)sBits[(b0 >> 5) + 1] << 32) | sBits[b0 >> 5];
+          const uint32_t mask = (uint32_t)(w2 >> (b0 & 31)) & 0xFFFFFFu;
+#pragma unroll
+          for (int i = 0; i < kMlaHalf; ++i) {
+            cur[i] = ((mask >> i) & 1u) ? cur[i] * p.scale_log2 : -INFINITY;
+            mhalf = fmaxf(mhalf, cur[i]);
+          }
+          sRed[((j & 1) * 2 + hf) * kMlaHeads + h] = mhalf;
+        }
+        // both halves of a head agree on the block max (and on whether to go on)
+        tc_fence_before();
+        if (!named_barrier_and(2, 128, ok)) break;
+        tc_fence_after();
+        // every owner thread has read inbox xb: re-arm it for block j+2 and hand
+        // the peer the credit (relaxed: the values are consumed)
+        if (announcer && j + kMlaXBufs < nblk) {
+          mbar_arrive_expect_tx(smem_u32(&xsfull[xb]), kMlaXsPayload);
+          mbar_arrive_remote_relaxed(xsfree_peer0 + (uint32_t)xb * 8u);
+        }
+        const float mblk =
+            fmaxf(sRed[((j & 1) * 2) * kMlaHeads + h], sRed[((j & 1) * 2 + 1) * kMlaHeads + h]);
+        // lazy rescale: move the reference max only when it grows by more than 8 (x256)
+        const bool grow = mblk > m_used + 8.0f;
+        const bool need_o = grow && m_used != -INFINITY;  // O already holds earlier blocks
+        const float f = need_o ? ex2_approx(m_used - mblk) : 1.0f;
+        if (__any_sync(0xffffffffu, need_o)) {
+          // O += P_{j-1} V_{j-1} must have finished before O is touched
+          if (!warp_wait(smem_u32(&kvempty[(j - 1) % kMlaStages]), ((j - 1) / kMlaStages) & 1, TO,
+                         abort_flag)) {
+            ok = false;
+          } else {
+            tc_fence_after();
+            rescale_o(f);
+          }
+        }
+        l *= f;
+        if (grow) m_used = mblk;
         // probabilities: bf16 for the PV product, fp32 for the normaliser
         uint32_t pk[kMlaHalf / 2];
         float lsum = 0.f;
@@ -504,30 +525,119 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           pk[i] = pack_bf16x2(p0, p1);
         }
         l += lsum;
-        // P_j over S_j: packed columns [12 hf, 12 hf + 12) of score buffer j
-        tmem_st8(tS(j) + hf * (kMlaHalf / 2) + lane_off, pk);
-        tmem_st4(tS(j) + hf * (kMlaHalf / 2) + 8 + lane_off, pk + 8);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(smem_u32(&pfull[j % kMlaSBufs]));
-      }
+        // P_j and the factor to the peer (its inbox xb is free once it has
+        // consumed block j-2 and returned the credit)
+        if (ok && j >= kMlaXBufs)
+          ok = warp_wait<true>(smem_u32(&xpfree[xb]), ((j / kMlaXBufs) - 1) & 1, TO, abort_flag);
+        if (ok) {
+          const uint32_t dst = xp_peer + xb * kMlaXpBytes + xp_off;
+          const uint32_t bar = xpfull_peer0 + xb * 8;
 #pragma unroll
-      for (int i = 0; i < kMlaHalf; ++i) cur[i] = nxt[i];
+          for (int c = 0; c < kMlaHalf / 8; ++c)
+            st_async_v4u(dst + c * kMlaXsChunk, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                         pk[4 * c + 3], bar);
+          if (hf == 0)
+            st_async_u32(xp_peer + xb * kMlaXpBytes + kMlaXpFactor + hl * 4, __float_as_uint(f),
+                         bar);
+        }
+        write_p(j, pk);
+      }
+    } else {
+      // ---------------------------------------------------- server of the peer's heads h
+      const uint32_t xs_peer = mapa_shared(smem_u32(sXs), peer);
+      const uint32_t xsfull_peer0 = mapa_shared(smem_u32(&xsfull[0]), peer);
+      const uint32_t xpfree_peer0 = mapa_shared(smem_u32(&xpfree[0]), peer);
+      // Block j's partial scores of these heads, from TMEM to the owner's inbox
+      // j % 2 (free from block 2 on once the owner consumed block j-2).
+      auto load_and_send = [&](int j) {
+        float v[kMlaHalf];
+        bool r = warp_wait(smem_u32(&sfull[j % kMlaSBufs]), (j / kMlaSBufs) & 1, TO, abort_flag);
+        if (r && j >= kMlaXBufs)
+          r = warp_wait<true>(smem_u32(&xsfree[j % kMlaXBufs]), ((j / kMlaXBufs) - 1) & 1, TO,
+                              abort_flag);
+        if (r) {
+          tc_fence_after();
+          load_s(j, v);
+          const uint32_t xb = (uint32_t)(j % kMlaXBufs);
+          const uint32_t dst = xs_peer + xb * kMlaXsBytes + xs_off;
+          const uint32_t bar = xsfull_peer0 + xb * 8;
+#pragma unroll
+          for (int c = 0; c < kMlaHalf / 4; ++c)
+            st_async_v4(dst + c * kMlaXsChunk, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3],
+                        bar);
+        }
+        return r;
+      };
+      if (nblk > 0) ok = load_and_send(0);
+      for (int j = 0; j < nblk; ++j) {
+        const int xb = j % kMlaXBufs;
+        // send ahead: block j+1 leaves before block j's P is awaited
+        if (ok && j + 1 < nblk) ok = load_and_send(j + 1);
+        uint32_t pk[kMlaHalf / 2];
+        float f = 1.0f;
+        if (ok) ok = warp_wait<true>(smem_u32(&xpfull[xb]), (j / kMlaXBufs) & 1, TO, abort_flag);
+        if (ok) {
+          const uint8_t* xr = sXp + xb * kMlaXpBytes + xp_off;
+#pragma unroll
+          for (int c = 0; c < kMlaHalf / 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xr + c * kMlaXsChunk);
+            pk[4 * c] = v.x;
+            pk[4 * c + 1] = v.y;
+            pk[4 * c + 2] = v.z;
+            pk[4 * c + 3] = v.w;
+          }
+          f = *reinterpret_cast<const float*>(sXp + xb * kMlaXpBytes + kMlaXpFactor + hl * 4);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kMlaHalf / 2; ++i) pk[i] = 0u;
+        }
+        tc_fence_before();
+        if (!named_barrier_and(3, 128, ok)) break;
+        tc_fence_after();
+        if (announcer && j + kMlaXBufs < nblk) {
+          mbar_arrive_expect_tx(smem_u32(&xpfull[xb]), kMlaXpPayload);
+          mbar_arrive_remote_relaxed(xpfree_peer0 + (uint32_t)xb * 8u);
+        }
+        // the owner moved its reference max: rescale these heads' O rows too
+        if (__any_sync(0xffffffffu, f != 1.0f)) {
+          if (!warp_wait(smem_u32(&kvempty[(j - 1) % kMlaStages]), ((j - 1) / kMlaStages) & 1, TO,
+                         abort_flag)) {
+            ok = false;
+          } else {
+            tc_fence_after();
+            rescale_o(f);
+          }
+        }
+        write_p(j, pk);
+      }
     }
-    // epilogue: every P.V product has finished once the last one has (in order)
+
+    // ------------------------------------------------------------------ epilogue
+    // every P.V product has finished once the last one has (in order)
     if (ok && nblk > 0)
       ok = warp_wait(smem_u32(&kvempty[(nblk - 1) % kMlaStages]), ((nblk - 1) / kMlaStages) & 1,
                      TO, abort_flag);
-    // the two halves' normalisers meet in exchange buffer 0: nothing arrives
-    // there any more (the peer's last block has been consumed), while the max
-    // swap slots may still be read by the other half of this head
-    float* sL = reinterpret_cast<float*>(sX);
-    sL[hf * kMlaHeads + h] = l;
+    if (own) sLh[hf * kMlaHeads + h] = l;
     tc_fence_before();
-    const bool all_ok = named_barrier_and(2, 256, ok);
+    const bool all_ok = named_barrier_and(4, 256, ok);
     tc_fence_after();
-    if (all_ok && nblk > 0) {
-      const float lt = sL[h] + sL[kMlaHeads + h];
+    float lt = 0.f;
+    bool lt_ok = all_ok;
+    if (own) {
+      lt = sLh[h] + sLh[kMlaHeads + h];
+      if (hf == 0) {
+        // the peer normalises its half of these heads' rows with the same sum
+        st_async_u32(mapa_shared(smem_u32(sLfin), peer) + hl * 4, __float_as_uint(lt),
+                     mapa_shared(smem_u32(lfull), peer));
+        if (all_ok)
+          p.lse[t * kMlaHeads + h] = lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994531f
+                                              : -INFINITY;
+      }
+    } else {
+      lt_ok = warp_wait<true>(smem_u32(lfull), 0, TO, abort_flag) && all_ok;
+      if (lt_ok) lt = reinterpret_cast<const float*>(sLfin)[hl];
+    }
+    if (lt_ok && nblk > 0) {
       const float inv = lt > 0.f ? 1.0f / lt : 0.f;
       __nv_bfloat16* orow = p.out + (t * kMlaHeads + h) * kMlaDv + d0 + hf * 128;
 #pragma unroll 1
@@ -543,9 +653,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                               pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
                               pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
       }
-      if (rank == 0 && hf == 0)
-        p.lse[t * kMlaHeads + h] = lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994531f
-                                            : -INFINITY;
     }
     if (h == 0 && hf == 0 && !seq_ok && rank == 0) report_error(kErrBounds);
     __syncwarp();
