@@ -2,7 +2,7 @@
 // lightning-indexer scores among the visible keys (DeepSeek-V3.2-Exp technical
 // report, zh translation, §1 "Architecture" and §2.1: S_t = Top-k(I_{t,:})).
 //
-// One CTA of 1024 threads per row. Scores are compared through an
+// One CTA of 512 threads per row, two per SM. Scores are compared through an
 // order-preserving 32-bit key (-0.0 maps to +0.0). The exact selection is a
 // radix select:
 //   find_kth   histograms of key bits [31:21], [20:10], [9:0] restricted to the
@@ -24,9 +24,11 @@
 
 namespace dsa {
 
-constexpr int kTopkThreads = 1024;
-constexpr int kTopkCacheElems = 40 * 1024;                     // 160 KB row cache
+constexpr int kTopkThreads = 512;                              // two CTAs (rows) per SM
+constexpr int kTopkCacheElems = 16 * 1024;                     // 64 KB: short row or candidates
 constexpr int kTopkCandCap = kTopkCacheElems / 2;              // candidates: key + position
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkBinsPerThread = 2048 / kTopkThreads;
 constexpr int kTopkSample = 2048;
 constexpr int kTopkSmemBytes = kTopkCacheElems * 4 + 2048 * 4 + 64 * 4 + kTopkSample * 4;
 
@@ -50,7 +52,7 @@ __device__ __forceinline__ uint32_t score_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive prefix sum over the 1024 threads of the block (uint32). Two barriers.
+// Exclusive prefix sum over the threads of the block (uint32). Two barriers.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot,
                                                          uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -63,14 +65,14 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    uint32_t w = warp_tot[lane];
+    uint32_t w = lane < kTopkWarps ? warp_tot[lane] : 0u;
     uint32_t wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       uint32_t n = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += n;
     }
-    warp_tot[lane] = wi - w;  // exclusive
+    if (lane < kTopkWarps) warp_tot[lane] = wi - w;  // exclusive
     if (lane == 31) *total = wi;
   }
   __syncthreads();
@@ -107,17 +109,22 @@ __device__ void find_kth(int n, uint32_t k, KeyAt key_at, uint32_t* hist, uint32
     }
     __syncthreads();
     // the bin holding the remaining-th largest key: bins walked from the top,
-    // two per thread (2047 - 2 tid, 2046 - 2 tid)
-    const int hi_bin = 2047 - 2 * tid, lo_bin = 2046 - 2 * tid;
-    const uint32_t c_hi = hi_bin < (int)nbins ? hist[hi_bin] : 0;
-    const uint32_t c_lo = lo_bin < (int)nbins ? hist[lo_bin] : 0;
-    const uint32_t above = block_exclusive_scan(c_hi + c_lo, misc, misc + 32);
-    if (above < remaining && remaining <= above + c_hi) {
-      misc[33] = hi_bin;
-      misc[34] = remaining - above;
-    } else if (above + c_hi < remaining && remaining <= above + c_hi + c_lo) {
-      misc[33] = lo_bin;
-      misc[34] = remaining - above - c_hi;
+    // kTopkBinsPerThread consecutive ones per thread (2047 - B tid - i)
+    uint32_t cnt[kTopkBinsPerThread], sum = 0;
+#pragma unroll
+    for (int i = 0; i < kTopkBinsPerThread; ++i) {
+      const int bin = 2047 - kTopkBinsPerThread * tid - i;
+      cnt[i] = bin < (int)nbins ? hist[bin] : 0u;
+      sum += cnt[i];
+    }
+    uint32_t above = block_exclusive_scan(sum, misc, misc + 32);
+#pragma unroll
+    for (int i = 0; i < kTopkBinsPerThread; ++i) {
+      if (above < remaining && remaining <= above + cnt[i]) {
+        misc[33] = 2047 - kTopkBinsPerThread * tid - i;
+        misc[34] = remaining - above;
+      }
+      above += cnt[i];
     }
     __syncthreads();
     const uint32_t d = misc[33];
@@ -174,7 +181,7 @@ __device__ void compact_topk(int n, uint32_t tau, uint32_t r_eq, KeyAt key_at, P
   }
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* cache = reinterpret_cast<float*>(smem_raw);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw + kTopkCacheElems * 4);
@@ -291,9 +298,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
   // (n <= 4k <= 8192 <= kTopkCacheElems; rows start 16-B aligned)
   {
     constexpr int kPer = 4 * kTopkThreads;
-    float4 v[2];
+    constexpr int kLoads = 8192 / kPer;  // n <= 4k <= 8192
+    float4 v[kLoads];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < kLoads; ++h) {
       const int e0 = h * kPer + 4 * tid;
       if (e0 + 3 < n) {
         v[h] = *reinterpret_cast<const float4*>(row + e0);
@@ -305,11 +313,11 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
       }
     }
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < kLoads; ++h) {
       const int e0 = h * kPer + 4 * tid;
       if (e0 < n) *reinterpret_cast<float4*>(cache + e0) = v[h];
     }
-    for (int e0 = 2 * kPer + 4 * tid; e0 < n; e0 += kPer)  // not reached for k <= 2048
+    for (int e0 = kLoads * kPer + 4 * tid; e0 < n; e0 += kPer)  // not reached for k <= 2048
       for (int u = 0; u < 4 && e0 + u < n; ++u) cache[e0 + u] = row[e0 + u];
     __syncthreads();
   }
