@@ -19,4 +19,7 @@ from .dsa_oracle import (  # noqa: F401
     dense_causal_mqa,
     resolve_kv_rows,
     dsa_forward,
+    indexer_kl_token,
+    sparse_indexer_kl,
+    dense_indexer_kl,
 )

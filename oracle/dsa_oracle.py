@@ -35,6 +35,11 @@ Readings where the pages are silent (each listed in the design doc):
   c_s[:512]; softmax with the given scale; LSE = ln sum_s exp(scale q.c_s).
   Entries of the index list outside [0, pos(t)] are ignored; an empty set gives
   o = 0 and LSE = -inf.
+* Indexer training target ([TR] §2.1, loss equations missing): the main
+  attention scores summed over the heads and L1-normalised along the sequence
+  are read as the head-mean of the per-head softmax over the set (a
+  distribution); the loss term of a row is KL(p || softmax(I)) over the set
+  (all visible keys in the dense warm-up, S_t in the sparse stage).
 
 Parity pins live in tests/test_oracle_*.py. Parity with values printed by the
 pages: unpinned (the pages print no worked values).
@@ -301,3 +306,65 @@ def dsa_forward(q_idx, w, k_idx, k_scale, q, kv, q_seq, q_pos, *, k, scale, d_v,
     o, lse = sparse_mla(q, kv, q_seq, q_pos, idx, scale, d_v, rows=rows,
                         block_table=block_table, page_size=page_size)
     return {"scores": scores, "idx": idx, "o": o, "lse": lse}
+
+
+# --------------------------------------------------------------------------------------
+# Indexer training target and KL loss ([TR] §2.1, both continued-pretraining stages)
+# --------------------------------------------------------------------------------------
+
+
+def indexer_kl_token(q_t, kv_rows, scores_sel, scale):
+    """KL loss term of one query token over a set of keys ([TR] §2.1).
+
+    q_t: [H, D]; kv_rows: [n, D] latent rows of the keys in the set; scores_sel:
+    [n] indexer scores I_{t,s} of the same keys. Reading of the pages (the loss
+    equations are missing images): the main attention of each head over the set
+    is a_h(s) = softmax_s(scale * q_h . c_s); the target p(s) sums a_h(s) over the
+    heads and L1-normalises over the set, i.e. p(s) = mean_h a_h(s); the model
+    distribution is softmax_s(I_{t,s}); the term is KL(p || softmax(I)) =
+    sum_s p(s) (ln p(s) - ln softmax(I)(s)), with 0 ln 0 = 0. All in fp64. An
+    empty set gives 0.
+    """
+    n = len(kv_rows)
+    if n == 0:
+        return 0.0
+    q64 = np.asarray(q_t, np.float64)
+    c = np.asarray(kv_rows, np.float64)
+    z = scale * (q64 @ c.T)                                  # [H, n]
+    z = z - np.max(z, axis=1, keepdims=True)
+    a = np.exp(z)
+    a = a / np.sum(a, axis=1, keepdims=True)                 # per-head softmax over the set
+    p = np.sum(a, axis=0)
+    p = p / np.sum(p)                                        # head-sum, L1-normalised
+    i64 = np.asarray(scores_sel, np.float64)
+    log_q = i64 - (np.max(i64) + np.log(np.sum(np.exp(i64 - np.max(i64)))))
+    nz = p > 0
+    return float(np.sum(p[nz] * (np.log(p[nz]) - log_q[nz])))
+
+
+def sparse_indexer_kl(q, kv, q_seq, q_pos, idx, scores, scale, *, rows=None, block_table=None,
+                      page_size=64):
+    """Sparse-stage KL term per query row ([TR] §2.1, sparse training stage): the
+    set is S_t, the entries of idx[r] inside [0, pos(t)] (as listed); scores[r]
+    is row t's indexer score row. Returns fp64 [R]; ``idx`` and ``scores`` are
+    indexed by the position of the row within ``rows``."""
+    T = q.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    out = np.zeros(len(rows))
+    for r, t in enumerate(rows):
+        b, pos = int(q_seq[t]), int(q_pos[t])
+        sel = [int(s) for s in idx[r] if 0 <= int(s) <= pos]
+        kv_rows = resolve_kv_rows(kv, b, sel, block_table, page_size) if sel else []
+        out[r] = indexer_kl_token(q[t], kv_rows, np.asarray(scores[r])[sel], scale)
+    return out
+
+
+def dense_indexer_kl(q, kv, q_seq, q_pos, scores, scale, *, rows=None, block_table=None,
+                     page_size=64):
+    """Dense warm-up KL term per query row ([TR] §2.1, dense warm-up stage): the
+    set is every visible key 0..pos(t)."""
+    T = q.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    idx = [np.arange(int(q_pos[t]) + 1) for t in rows]
+    return sparse_indexer_kl(q, kv, q_seq, q_pos, idx, scores, scale, rows=rows,
+                             block_table=block_table, page_size=page_size)
