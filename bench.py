@@ -94,6 +94,11 @@ def algorithmic_work(p: synth.Problem, k: int = K_SEL) -> dict:
         "indexer": {"bytes": idx_bytes, "flop": idx_flop, "flop_dtype": "fp8"},
         "topk": {"bytes": topk_bytes, "flop": 0, "flop_dtype": None},
         "sparse_mla": {"bytes": mla_bytes, "flop": mla_flop, "flop_dtype": "bf16"},
+        # indexer KL loss term: Q, LSE, idx, the score and latent row of every
+        # selected key per row; the 128-head score of every selected key
+        "indexer_kl": {"bytes": T * (128 * 576 * 2 + 128 * 4 + 4 * k + 4) +
+                       (1152 + 4) * int(n_sel.sum()),
+                       "flop": 2 * 128 * 576 * int(n_sel.sum()), "flop_dtype": "bf16"},
     }
 
 
@@ -202,7 +207,7 @@ class Runner:
     """Holds the device buffers of one workload and runs one step of the path
     through the library's stage calls (the same launches dsa_forward makes)."""
 
-    def __init__(self, p: synth.Problem, k: int = K_SEL):
+    def __init__(self, p: synth.Problem, k: int = K_SEL, with_kl: bool = False):
         from sparse_attention_05_b200 import dsa
         self.dsa = dsa
         self.p = p
@@ -221,6 +226,12 @@ class Runner:
         self.out = torch.empty(T, 128, 512, dtype=torch.bfloat16, device=p.q.device)
         self.lse = torch.empty(T, 128, dtype=torch.float32, device=p.q.device)
         self.launches_per_step = 2 * len(self.chunks) + 1
+        self.with_kl = with_kl
+        if with_kl:
+            if len(self.chunks) > 1:
+                raise SystemExit("--kl needs every score row in one chunk (not this workload)")
+            self.kl = torch.empty(T, dtype=torch.float32, device=p.q.device)
+            self.launches_per_step += 1
 
     def step(self, ev=None):
         d, p = self.dsa, self.p
@@ -242,6 +253,13 @@ class Runner:
                              lse=self.lse)
         if ev is not None:
             ev["sparse_mla"].append(_record())
+        if self.with_kl:  # the indexer's KL loss term over the selected sets
+            if ev is not None:
+                ev["indexer_kl"].append(_record())
+            d.dsa_indexer_kl(p.q, p.kv, self.kv, p.q_per_seq, self.idx, p.scale, self.lse,
+                             self.scores, kl=self.kl)
+            if ev is not None:
+                ev["indexer_kl"].append(_record())
 
 
 def _record():
@@ -477,6 +495,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--kl", action="store_true",
+                    help="also run the indexer KL loss term (training target) every step")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the decode batch (small cases for profiler captures)")
     ap.add_argument("--soak-s", type=float, default=1.0,
@@ -489,7 +509,7 @@ def main(argv=None):
 
     world, rank, local = dist_setup(args.gpus)
     p = make_problem(args.workload, "cuda", seed_offset=rank, batch=args.batch)
-    r = Runner(p)
+    r = Runner(p, with_kl=args.kl)
     work = algorithmic_work(p)
     peaks = load_peaks()
 
@@ -504,6 +524,8 @@ def main(argv=None):
     barrier(world)
     torch.cuda.synchronize()
     ev = {"indexer": [], "topk": [], "sparse_mla": []}
+    if args.kl:
+        ev["indexer_kl"] = []
     start = _record()
     for _ in range(args.steps):
         r.step(ev)
@@ -539,7 +561,8 @@ def main(argv=None):
 
     if rank == 0:
         cfg = {"workload": args.workload, **WORKLOADS[args.workload],
-               **({"batch": args.batch} if args.batch else {}), "k": K_SEL,
+               **({"batch": args.batch} if args.batch else {}),
+               **({"indexer_kl": True} if args.kl else {}), "k": K_SEL,
                "heads": 128, "d_qk": 576, "d_v": 512, "h_idx": 64, "d_idx": 128,
                "query_rows_per_gpu": p.num_q,
                "l2": "inputs larger than L2 (no flush)",

@@ -137,6 +137,26 @@ DSA_API dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv_cache, con
 
 /* Bytes of device workspace dsa_forward needs for this geometry (0 on a
  * geometry the library rejects). */
+/* Indexer training target and KL loss term (report §2.1: the main attention summed
+ * over all heads and L1-normalised along the sequence is the target p_{t,:}; the
+ * indexer is trained with KL(p_{t,:} || Softmax(I_{t,:})), over every visible key in
+ * the dense warm-up stage and over S_t in the sparse stage). For query row t and the
+ * set S of entries of idx[t] inside [0, pos(t)] (as listed):
+ *   a_h(s) = exp(scale q_{t,h} . c_s - lse[t][h])   (head h's attention over S)
+ *   p(s)   = mean_h a_h(s),   q(s) = softmax_{s in S}(I_{t,s})
+ *   kl[r]  = sum_{s in S} p(s) (ln p(s) - ln q(s))    (0 for an empty S)
+ *  q, kv, the caches' geometry and idx as for dsa_sparse_mla_fwd; k in [1, 2^20]
+ *         (the dense stage passes every visible position)
+ *  lse    fp32 [T][128] the LSE dsa_sparse_mla_fwd wrote for the same idx and scale
+ *  scores fp32 [batch * row_count][ld] indexer score rows of the window (as
+ *         dsa_indexer_scores writes them); ld >= max_ctx
+ *  kl     fp32 [batch * row_count] out, one term per row of the window.
+ * Shapes: 128 heads x 576-d latents only. */
+DSA_API dsa_status_t dsa_indexer_kl(const void* q, const void* kv_cache, const dsa_kv_desc_t* kv,
+                                    const dsa_q_desc_t* qd, const int32_t* idx, int32_t k,
+                                    float scale, const float* lse, const float* scores,
+                                    int64_t ld, float* kl, dsa_stream_t stream);
+
 DSA_API size_t dsa_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k);
 
 /* The whole forward: indexer scores -> top-k -> sparse MLA, on `stream`.

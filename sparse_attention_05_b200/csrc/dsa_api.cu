@@ -15,6 +15,7 @@
 #include "topk.cuh"
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
+#include "indexer_kl.cuh"
 
 using namespace dsa;
 
@@ -229,6 +230,45 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
   return cuda_status(cudaLaunchKernelEx(&cfg, sparse_mla_kernel, p, tm));
 }
 
+// ---- indexer KL launch -------------------------------------------------------------
+dsa_status_t launch_indexer_kl(const void* q, const void* kv_cache, const Geometry& g,
+                               const int32_t* idx, int k, float scale, const float* lse,
+                               const float* scores, int64_t ld, float* kl, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(indexer_kl_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kKlSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  KlParams p{};
+  p.kv = reinterpret_cast<const uint8_t*>(kv_cache);
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.idx = idx;
+  p.lse = lse;
+  p.scores = scores;
+  p.block_table = g.block_table;
+  p.seqlens = g.seqlens;
+  p.kl = kl;
+  p.ld = ld;
+  p.k = k;
+  p.batch = g.batch;
+  p.max_ctx = g.max_ctx;
+  p.q_per_seq = g.q_per_seq;
+  p.row_begin = g.row_begin;
+  p.row_count = g.row_count;
+  p.paged = g.layout == DSA_KV_PAGED;
+  p.page_size = g.page_size;
+  p.max_pages = g.max_pages;
+  p.num_pages = g.num_pages;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+  const int64_t grid = (int64_t)g.batch * g.row_count;
+  if (grid == 0) return DSA_OK;
+  indexer_kl_kernel<<<(unsigned)grid, kKlThreads, kKlSmemBytes, stream>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
 // ---- dsa_forward workspace plan --------------------------------------------------------
 constexpr int64_t kScoreBudgetBytes = 2ll << 30;  // bound on one chunk of score rows
 
@@ -380,6 +420,22 @@ dsa_status_t dsa_forward_noalloc(const void* q_idx, const float* w, const void* 
   if (st != DSA_OK) return st;
   return dsa_forward(q_idx, w, k_idx, k_scale, q, kv_cache, kv, qd, k, scale, scratch,
                      kStaticScratchBytes, idx_out, out, lse, stream);
+}
+
+dsa_status_t dsa_indexer_kl(const void* q, const void* kv_cache, const dsa_kv_desc_t* kv,
+                            const dsa_q_desc_t* qd, const int32_t* idx, int32_t k, float scale,
+                            const float* lse, const float* scores, int64_t ld, float* kl,
+                            dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !kv_cache || !idx || !lse || !scores || !kl) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_cache)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > (1 << 20)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (ld < g.max_ctx) return DSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !(scale < 1e30f)) return DSA_ERR_INVALID_ARG;
+  return launch_indexer_kl(q, kv_cache, g, idx, k, scale, lse, scores, ld, kl,
+                           (cudaStream_t)stream);
 }
 
 dsa_status_t dsa_selftest_wait_timeout(dsa_stream_t stream) {

@@ -60,6 +60,9 @@ SIGNATURES = {
                                 ctypes.POINTER(QDescC), ctypes.c_int32, _P, _P]),
     "dsa_sparse_mla_fwd": (ctypes.c_int, [_P, _P, ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
                                           _P, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
+    "dsa_indexer_kl": (ctypes.c_int, [_P, _P, ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
+                                      _P, ctypes.c_int32, ctypes.c_float, _P, _P, ctypes.c_int64,
+                                      _P, _P]),
     "dsa_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
                                              ctypes.c_int32]),
     "dsa_forward": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.POINTER(KvDescC),
@@ -201,6 +204,21 @@ def dsa_sparse_mla_fwd(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale: fl
                                     _ptr(idx), idx.shape[1], float(scale), _ptr(out), _ptr(lse),
                                     _stream(stream)), "dsa_sparse_mla_fwd")
     return out, lse
+
+
+def dsa_indexer_kl(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale: float, lse, scores,
+                   kl: Optional[torch.Tensor] = None, rows=None, stream=None) -> torch.Tensor:
+    """KL(p || softmax(I)) per row of the window (include/dsa.h): idx [T][k], lse
+    [T][128] from dsa_sparse_mla_fwd, scores [batch * window rows][ld]."""
+    T = q.shape[0]
+    if kl is None:
+        kl = torch.empty(kv.batch * _window(kv, q_per_seq, rows), dtype=torch.float32,
+                         device=q.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    _check(lib().dsa_indexer_kl(_ptr(q), _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd),
+                                _ptr(idx), idx.shape[1], float(scale), _ptr(lse), _ptr(scores),
+                                scores.shape[1], _ptr(kl), _stream(stream)), "dsa_indexer_kl")
+    return kl
 
 
 def dsa_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None) -> int:
