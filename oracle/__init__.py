@@ -22,4 +22,8 @@ from .dsa_oracle import (  # noqa: F401
     indexer_kl_token,
     sparse_indexer_kl,
     dense_indexer_kl,
+    mla_up_project,
+    mha_head_attention,
+    masked_mha,
+    absorb_mha_query,
 )

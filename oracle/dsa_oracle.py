@@ -40,6 +40,14 @@ Readings where the pages are silent (each listed in the design doc):
   are read as the head-mean of the per-head softmax over the set (a
   distribution); the loss term of a row is KL(p || softmax(I)) over the set
   (all visible keys in the dense warm-up, S_t in the sparse stage).
+* MLA in MHA mode ([TR] Appendix A, Fig. 4 missing) and its masked form for
+  short prefill ([TR] §3): per head h the key is [W^UK_h c_s[:512] ; c_s[512:]]
+  (the 64 rope dims shared by all heads) and the value W^UV_h c_s[:512], with
+  128 nope query/key dims and 128 value dims per head (the pages give no
+  per-head sizes); the decompressed keys and values are held in bf16. The mask
+  of row t is its selected set S_t (plain causal when every visible key is
+  selected); the softmax scale is the one MQA mode uses, so that both modes
+  compute the same logits.
 
 Parity pins live in tests/test_oracle_*.py. Parity with values printed by the
 pages: unpinned (the pages print no worked values).
@@ -368,3 +376,92 @@ def dense_indexer_kl(q, kv, q_seq, q_pos, scores, scale, *, rows=None, block_tab
     idx = [np.arange(int(q_pos[t]) + 1) for t in rows]
     return sparse_indexer_kl(q, kv, q_seq, q_pos, idx, scores, scale, rows=rows,
                              block_table=block_table, page_size=page_size)
+
+
+# --------------------------------------------------------------------------------------
+# MLA in MHA mode and the masked-MHA emulation of DSA ([TR] Appendix A, Fig. 4;
+# [TR] §3 "Inference cost": short-sequence prefill runs a masked MHA mode)
+# --------------------------------------------------------------------------------------
+
+
+def mla_up_project(c_rows, w_uk_h, w_uv_h, *, round_kv=True):
+    """MHA-mode key and value of one head for latent rows ``c_rows`` [n, d_c + d_r].
+
+    k_{h,s} = [W^UK_h c_s[:d_c] ; c_s[d_c:]] (the rope part is shared by all
+    heads: it does not pass through the up-projection) and v_{h,s} =
+    W^UV_h c_s[:d_c], with w_uk_h [d_n, d_c] and w_uv_h [d_hv, d_c]. Computed in
+    fp64; with ``round_kv`` both are rounded to bf16, the format in which the
+    MHA mode holds its decompressed keys and values. Returns (k [n, d_n + d_r],
+    v [n, d_hv]) as fp64.
+    """
+    c = np.asarray(c_rows, np.float64)
+    uk = np.asarray(w_uk_h, np.float64)
+    uv = np.asarray(w_uv_h, np.float64)
+    d_c = uk.shape[1]
+    k = np.concatenate([c[:, :d_c] @ uk.T, c[:, d_c:]], axis=1)
+    v = c[:, :d_c] @ uv.T
+    if round_kv:
+        k = bf16_round(k).astype(np.float64)
+        v = bf16_round(v).astype(np.float64)
+    return k, v
+
+
+def mha_head_attention(q_th, k, v, scale):
+    """Softmax attention of one head's query ``q_th`` [d_qk] over keys k [n, d_qk]
+    and values v [n, d_hv]: (o [d_hv], lse) in fp64; n == 0 gives (0, -inf)."""
+    if len(k) == 0:
+        return np.zeros(v.shape[1]), -np.inf
+    z = scale * (k @ np.asarray(q_th, np.float64))
+    m = np.max(z)
+    lse = m + np.log(np.sum(np.exp(z - m)))
+    return np.exp(z - lse) @ v, lse
+
+
+def masked_mha(q, kv, q_seq, q_pos, idx, scale, w_uk, w_uv, *, rows=None, block_table=None,
+               page_size=64, round_kv=True):
+    """Masked MHA emulation of DSA for query rows ``rows`` (default: all).
+
+    q: [T, H, d_n + d_r] MHA-mode queries (q^C_{t,h} ; q^R_{t,h}); kv: the latent
+    cache; w_uk: [H, d_n, d_c]; w_uv: [H, d_hv, d_c]. Row t of head h attends,
+    with softmax scale ``scale``, over the set {s in idx[r] : 0 <= s <= pos(t)}
+    (a set: an entry listed twice counts once) or, when ``idx`` is None, over every
+    visible key 0..pos(t) (plain causal MHA). Keys and values come from
+    mla_up_project. Returns (o fp64 [R, H, d_hv], lse fp64 [R, H]); ``idx`` is
+    indexed by the position of the row within ``rows``.
+
+    Heads are independent, so the loop runs head by head over the rows of each
+    sequence, up-projecting the sequence's visible latent rows once per head.
+    """
+    T, H = q.shape[0], q.shape[1]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    d_hv = np.asarray(w_uv).shape[1]
+    o = np.zeros((len(rows), H, d_hv))
+    lse = np.full((len(rows), H), -np.inf)
+    sets = []
+    for r, t in enumerate(rows):
+        pos = int(q_pos[t])
+        if idx is None:
+            sets.append(np.arange(pos + 1))
+        else:
+            sets.append(np.unique([int(s) for s in idx[r] if 0 <= int(s) <= pos]).astype(np.int64))
+    for b in sorted({int(q_seq[t]) for t in rows}):
+        mine = [r for r, t in enumerate(rows) if int(q_seq[t]) == b]
+        n_keys = max(int(q_pos[rows[r]]) for r in mine) + 1
+        c = resolve_kv_rows(kv, b, list(range(n_keys)), block_table, page_size)
+        for h in range(H):
+            k_h, v_h = mla_up_project(c, w_uk[h], w_uv[h], round_kv=round_kv)
+            for r in mine:
+                s = sets[r]
+                o[r, h], lse[r, h] = mha_head_attention(q[rows[r], h], k_h[s], v_h[s], scale)
+    return o, lse
+
+
+def absorb_mha_query(q_mha, w_uk):
+    """The MHA-to-MQA conversion of a query ([TR] Appendix A): per head,
+    q~_h = [W^UK_h^T q^C_h ; q^R_h], so that q~_h . c_s = q_h . k_{h,s} for the
+    unrounded MHA-mode key. q_mha: [T, H, d_n + d_r]; w_uk: [H, d_n, d_c]."""
+    q64 = np.asarray(q_mha, np.float64)
+    uk = np.asarray(w_uk, np.float64)
+    d_n = uk.shape[1]
+    nope = np.einsum("thn,hnc->thc", q64[:, :, :d_n], uk)
+    return np.concatenate([nope, q64[:, :, d_n:]], axis=2)

@@ -220,3 +220,35 @@ def sample_rows(T: int, n: int, seed: int, must=()) -> torch.Tensor:
 
 def pages_needed(seqlens: torch.Tensor, page_size: int) -> int:
     return int(sum(math.ceil(int(s) / page_size) for s in seqlens.tolist()))
+
+
+@dataclasses.dataclass
+class MhaInputs:
+    """Extra inputs of MLA's MHA mode for a Problem's query rows and latent cache.
+
+    q_mha [T, H, d_n + d_r] bf16  per-head queries (128 nope dims, then the 64 rope dims)
+    w_uk  [H, d_n, d_c]     bf16  key up-projection of each head (d_c = 512 latent dims)
+    w_uv  [H, d_hv, d_c]    bf16  value up-projection of each head
+    """
+    q_mha: torch.Tensor
+    w_uk: torch.Tensor
+    w_uv: torch.Tensor
+
+    def to(self, device) -> "MhaInputs":
+        return MhaInputs(self.q_mha.to(device), self.w_uk.to(device), self.w_uv.to(device))
+
+
+MHA_NOPE = 128   # nope query/key dims per head
+MHA_ROPE = 64    # rope dims (shared key part)
+MHA_DV = 128     # value dims per head
+
+
+def mha_inputs(p: Problem, seed: int, device="cpu") -> MhaInputs:
+    """q_mha ~ N(0,1) and random-init up-projections W ~ N(0, 1/d_c), all bf16
+    (no trained weights: the kernels' cost and numerics do not depend on them)."""
+    g = _gen(seed, device)
+    H, d_c = p.dims.heads, p.dims.d_v
+    q_mha = _bf16((p.num_q, H, MHA_NOPE + MHA_ROPE), g, device)
+    w_uk = _bf16((H, MHA_NOPE, d_c), g, device, std=d_c ** -0.5)
+    w_uv = _bf16((H, MHA_DV, d_c), g, device, std=d_c ** -0.5)
+    return MhaInputs(q_mha, w_uk, w_uv)
