@@ -135,8 +135,6 @@ DSA_API dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv_cache, con
                                 const dsa_q_desc_t* qd, const int32_t* idx, int32_t k,
                                 float scale, void* out, float* lse, dsa_stream_t stream);
 
-/* Bytes of device workspace dsa_forward needs for this geometry (0 on a
- * geometry the library rejects). */
 /* Indexer training target and KL loss term (report §2.1: the main attention summed
  * over all heads and L1-normalised along the sequence is the target p_{t,:}; the
  * indexer is trained with KL(p_{t,:} || Softmax(I_{t,:})), over every visible key in
@@ -157,6 +155,8 @@ DSA_API dsa_status_t dsa_indexer_kl(const void* q, const void* kv_cache, const d
                                     float scale, const float* lse, const float* scores,
                                     int64_t ld, float* kl, dsa_stream_t stream);
 
+/* Bytes of device workspace dsa_forward needs for this geometry (0 on a
+ * geometry the library rejects). */
 DSA_API size_t dsa_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k);
 
 /* The whole forward: indexer scores -> top-k -> sparse MLA, on `stream`.
@@ -199,6 +199,82 @@ DSA_API dsa_status_t dsa_forward_noalloc(const void* q_idx, const float* w, cons
                                          const dsa_q_desc_t* qd, int32_t k, float scale,
                                          int32_t* idx_out, void* out, float* lse,
                                          dsa_stream_t stream);
+
+/* ---- MLA in MHA mode: the masked-MHA emulation of DSA for short prefill ----------
+ * Report Appendix A (Fig. 4): MLA runs in an MHA mode (training, prefill) or an MQA
+ * mode (decode); report §3 "Inference cost": for short-sequence prefill a masked MHA
+ * mode emulates DSA. Per head h (128 heads) the MHA-mode key of token s is
+ * k_{h,s} = [W^UK_h c_s[0:512] ; c_s[512:576]] (128 nope dims, then the 64 rope
+ * dims every head shares) and its value v_{h,s} = W^UV_h c_s[0:512] (128 dims);
+ * the query of row t is q_{t,h} = [q^C (128) ; q^R (64)]. Row t attends over its
+ * selected set S_t (every visible key when pos(t) + 1 <= k): the result equals
+ * the MQA-mode sparse MLA of the absorbed query [W^UK_h^T q^C ; q^R] followed by
+ * W^UV_h on its output, with the same LSE. */
+
+/* Decompresses the latent cache into MHA-mode keys and values (bf16, fp32
+ * accumulation). For every sequence b, head h and token s < seqlen[b]:
+ *  k_nope bf16 [batch][128][ctx_pad][128] out: W^UK_h c_s[0:512]
+ *  k_rope bf16 [batch][ctx_pad][64]      out: c_s[512:576]
+ *  v      bf16 [batch][128][ctx_pad][128] out: W^UV_h c_s[0:512]
+ * Slots s in [seqlen, round_up(seqlen, 128)) are written as zeros; later slots are
+ * not written.
+ *  kv_cache bf16 latent cache as for dsa_sparse_mla_fwd (contiguous or paged)
+ *  w_uk, w_uv bf16 [128][128][512]: row d of head h is the weight vector of output
+ *           dim d (W^UK_h and W^UV_h, row-major)
+ *  ctx_pad  a multiple of 128, >= max_ctx rounded up to 128; batch * 128 * ctx_pad
+ *           must stay below 2^31. */
+DSA_API dsa_status_t dsa_mla_up_project(const void* kv_cache, const void* w_uk, const void* w_uv,
+                                        const dsa_kv_desc_t* kv, void* k_nope, void* k_rope,
+                                        void* v, int64_t ctx_pad, dsa_stream_t stream);
+
+/* Selection bitmask of the window's rows: for every row t of the window with
+ * pos(t) + 1 > k, bit s of mask[t] (word s / 32, bit s % 32) is set iff s is an
+ * entry of idx[t] inside [0, pos(t)]; the words of the 128-key tiles up to pos(t)
+ * are written, the rest of the row is not. Rows with pos(t) + 1 <= k select every
+ * visible key and are not written.
+ *  idx  int32 [T][k] (as dsa_topk writes it)
+ *  mask uint32 [T][mask_ld] out, 16-byte aligned; mask_ld a multiple of 4 and
+ *       >= 4 * ceil(max_ctx / 128) (at most 58112 words). */
+DSA_API dsa_status_t dsa_selection_mask(const int32_t* idx, int32_t k, const dsa_kv_desc_t* kv,
+                                        const dsa_q_desc_t* qd, uint32_t* mask, int64_t mask_ld,
+                                        dsa_stream_t stream);
+
+/* Masked MHA over the decompressed keys and values (flash attention, 128-row by
+ * 128-key tiles on the tensor cores, P rounded to bf16):
+ *  q_mha bf16 [T][128][192] MHA-mode queries (128 nope dims, then 64 rope dims)
+ *  k_nope, k_rope, v, ctx_pad as dsa_mla_up_project wrote them
+ *  mask  NULL: every row attends over all of 0..pos(t) (causal MHA). Otherwise
+ *        rows with pos(t) + 1 > k attend over the keys whose bit is set in
+ *        mask[t] (dsa_selection_mask), the others over 0..pos(t).
+ *  out   bf16 [T][128][128] out: o_{t,h} = sum_s softmax_s(scale q_{t,h} . k_{h,s}) v_{h,s}
+ *  lse   fp32 [T][128] out: ln sum_s exp(scale q_{t,h} . k_{h,s}); a row with no
+ *        admitted key gets o = 0 and lse = -inf. */
+DSA_API dsa_status_t dsa_masked_mha(const void* q_mha, const void* k_nope, const void* k_rope,
+                                    const void* v, int64_t ctx_pad, const dsa_kv_desc_t* kv,
+                                    const dsa_q_desc_t* qd, const uint32_t* mask,
+                                    int64_t mask_ld, int32_t k, float scale, void* out,
+                                    float* lse, dsa_stream_t stream);
+
+/* Bytes of device workspace dsa_mha_prefill needs (0 on a rejected geometry). */
+DSA_API size_t dsa_mha_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k);
+
+/* Short-prefill DSA in MHA mode: indexer scores and top-k for the rows with more
+ * than k visible keys (when seqlens is NULL the rows with pos(t) + 1 <= k are
+ * skipped; with a seqlens array every row of the window is scored), their
+ * selection masks, the up-projection of the latent cache, then the masked MHA.
+ * Inputs as for dsa_forward plus q_mha, w_uk and w_uv; out and lse as for
+ * dsa_masked_mha. `workspace` (256-byte aligned) holds the indices (unless idx_out
+ * is given), the masks, the decompressed keys and values and a chunk of score
+ * rows; dsa_mha_workspace_size() bytes give the largest chunk, smaller
+ * workspaces down to one score row per sequence are accepted. idx_out, when not
+ * NULL, receives the selection of every row of the window. */
+DSA_API dsa_status_t dsa_mha_prefill(const void* q_idx, const float* w, const void* k_idx,
+                                     const float* k_scale, const void* q_mha,
+                                     const void* kv_cache, const void* w_uk, const void* w_uv,
+                                     const dsa_kv_desc_t* kv, const dsa_q_desc_t* qd, int32_t k,
+                                     float scale, void* workspace, size_t workspace_bytes,
+                                     int32_t* idx_out, void* out, float* lse,
+                                     dsa_stream_t stream);
 
 /* Synchronizes `stream`, then returns and clears the device error word
  * (DSA_OK when no kernel reported a problem since the last call). */

@@ -14,7 +14,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdsa.so")
 SOURCES = ["dsa_api.cu"]
-HEADERS = ["ptx.cuh", "topk.cuh", "indexer.cuh", "sparse_mla.cuh", "indexer_kl.cuh"]
+HEADERS = ["ptx.cuh", "topk.cuh", "indexer.cuh", "sparse_mla.cuh", "indexer_kl.cuh",
+           "mha_prefill.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

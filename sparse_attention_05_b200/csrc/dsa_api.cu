@@ -16,6 +16,7 @@
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
 #include "indexer_kl.cuh"
+#include "mha_prefill.cuh"
 
 using namespace dsa;
 
@@ -297,6 +298,158 @@ ForwardPlan plan_forward(const Geometry& g, int k, bool need_idx) {
   return f;
 }
 
+// ---- MHA mode: up-projection, selection mask, masked MHA --------------------------------
+// 3-D row-major tensor [d2][d1][d0] with 128-byte swizzled boxes.
+dsa_status_t make_tmap_3d(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                          int elem_bytes, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                          uint32_t b1, uint32_t b2) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return DSA_ERR_CUDA;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * elem_bytes, d0 * d1 * elem_bytes};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(tm, dtype, 3, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
+}
+
+struct MhaPlan {
+  int key_tiles;
+  int64_t ctx_pad;      // key slots per (sequence, head) in the decompressed tensors
+  int64_t mask_ld;      // words per selection-mask row
+  size_t kn_bytes, kr_bytes, v_bytes, mask_bytes;
+};
+
+MhaPlan plan_mha(const Geometry& g) {
+  MhaPlan m;
+  m.key_tiles = (g.max_ctx + kMhaTile - 1) / kMhaTile;
+  m.ctx_pad = (int64_t)m.key_tiles * kMhaTile;
+  m.mask_ld = (int64_t)m.key_tiles * 4;
+  m.kn_bytes = align256((size_t)g.batch * kMhaHeads * m.ctx_pad * kMhaDn * 2);
+  m.kr_bytes = align256((size_t)g.batch * m.ctx_pad * kMhaDr * 2);
+  m.v_bytes = align256((size_t)g.batch * kMhaHeads * m.ctx_pad * kMhaDv * 2);
+  m.mask_bytes = align256((size_t)g.num_q * m.mask_ld * 4);
+  return m;
+}
+
+// every decompressed row index of the tensor maps must fit in int32
+bool mha_fits(const Geometry& g, int64_t ctx_pad) {
+  return (int64_t)g.batch * kMhaHeads * ctx_pad < (1ll << 31);
+}
+
+dsa_status_t launch_up_proj(const void* kv_cache, const void* w_uk, const void* w_uv,
+                            const Geometry& g, void* k_nope, void* k_rope, void* v,
+                            int64_t ctx_pad, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(mla_up_proj_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kUpSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  CUtensorMap tm_lat, tm_uk, tm_uv;
+  dsa_status_t st = make_tmap_2d(&tm_lat, kv_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMhaLat,
+                                 (uint64_t)g.cache_rows, 64, 64);
+  if (st == DSA_OK)
+    st = make_tmap_2d(&tm_uk, w_uk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMhaDc,
+                      (uint64_t)kMhaHeads * kMhaDn, 64, kMhaDn);
+  if (st == DSA_OK)
+    st = make_tmap_2d(&tm_uv, w_uv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMhaDc,
+                      (uint64_t)kMhaHeads * kMhaDv, 64, kMhaDv);
+  if (st != DSA_OK) return st;
+  UpProjParams p{};
+  p.block_table = g.block_table;
+  p.seqlens = g.seqlens;
+  p.kv = reinterpret_cast<const __nv_bfloat16*>(kv_cache);
+  p.k_nope = reinterpret_cast<__nv_bfloat16*>(k_nope);
+  p.k_rope = reinterpret_cast<__nv_bfloat16*>(k_rope);
+  p.v = reinterpret_cast<__nv_bfloat16*>(v);
+  p.ctx_pad = ctx_pad;
+  p.batch = g.batch;
+  p.max_ctx = g.max_ctx;
+  p.q_per_seq = g.q_per_seq;
+  p.paged = g.layout == DSA_KV_PAGED;
+  p.page_size = g.page_size;
+  p.max_pages = g.max_pages;
+  p.num_pages = g.num_pages;
+  p.key_tiles = (g.max_ctx + kMhaTile - 1) / kMhaTile;
+  p.timeout_ns = g_timeout_ns.load();
+  const int64_t items = (int64_t)g.batch * p.key_tiles * kMhaHeads;
+  const int grid = (int)std::min<int64_t>(items, num_sms());
+  mla_up_proj_kernel<<<grid, kUpThreads, kUpSmemBytes, stream>>>(p, tm_lat, tm_uk, tm_uv);
+  return cuda_status(cudaGetLastError());
+}
+
+dsa_status_t launch_selection_mask(const int32_t* idx, int k, const Geometry& g, int row_begin,
+                                   int row_count, uint32_t* mask, int64_t mask_ld,
+                                   cudaStream_t stream) {
+  const size_t smem = (size_t)mask_ld * 4;
+  if (smem > 227 * 1024) return DSA_ERR_UNSUPPORTED_SHAPE;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(selection_mask_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  MaskParams p{idx, g.seqlens, mask, mask_ld, k, g.batch, g.max_ctx, g.q_per_seq, row_begin,
+               row_count};
+  const int64_t grid = (int64_t)g.batch * row_count;
+  if (grid == 0) return DSA_OK;
+  selection_mask_kernel<<<(unsigned)grid, kMaskThreads, smem, stream>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+dsa_status_t launch_masked_mha(const void* q_mha, const void* k_nope, const void* k_rope,
+                               const void* v, int64_t ctx_pad, const Geometry& g,
+                               const uint32_t* mask, int64_t mask_ld, int k, float scale,
+                               void* out, float* lse, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(masked_mha_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kFaSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  CUtensorMap tm_q, tm_kn, tm_kr, tm_v;
+  const uint64_t kv_rows = (uint64_t)g.batch * kMhaHeads * ctx_pad;
+  dsa_status_t st = make_tmap_3d(&tm_q, q_mha, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMhaDqk,
+                                 kMhaHeads, (uint64_t)g.num_q, 64, 1, kMhaTile);
+  if (st == DSA_OK)
+    st = make_tmap_2d(&tm_kn, k_nope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMhaDn, kv_rows, 64,
+                      kMhaTile);
+  if (st == DSA_OK)
+    st = make_tmap_2d(&tm_kr, k_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMhaDr,
+                      (uint64_t)g.batch * ctx_pad, 64, kMhaTile);
+  if (st == DSA_OK)
+    st = make_tmap_2d(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMhaDv, kv_rows, 64,
+                      kMhaTile);
+  if (st != DSA_OK) return st;
+  MhaParams p{};
+  p.seqlens = g.seqlens;
+  p.mask = mask;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.ctx_pad = ctx_pad;
+  p.mask_ld = mask_ld;
+  p.batch = g.batch;
+  p.max_ctx = g.max_ctx;
+  p.q_per_seq = g.q_per_seq;
+  p.row_begin = g.row_begin;
+  p.row_count = g.row_count;
+  p.row_blocks = (g.row_count + kMhaTile - 1) / kMhaTile;
+  p.k = k;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_timeout_ns.load();
+  const int64_t grid = (int64_t)p.row_blocks * g.batch * kMhaHeads;
+  if (grid == 0) return DSA_OK;
+  masked_mha_kernel<<<(unsigned)grid, kFaThreads, kFaSmemBytes, stream>>>(p, tm_q, tm_kn, tm_kr,
+                                                                           tm_v);
+  return cuda_status(cudaGetLastError());
+}
+
 // ---- scratch for the allocation-free forward ------------------------------------------
 // A fixed device array that every device loading this library holds until exit.
 // Host code must not use the symbol's host-side address: the device address is
@@ -436,6 +589,143 @@ dsa_status_t dsa_indexer_kl(const void* q, const void* kv_cache, const dsa_kv_de
   if (!(scale > 0.f) || !(scale < 1e30f)) return DSA_ERR_INVALID_ARG;
   return launch_indexer_kl(q, kv_cache, g, idx, k, scale, lse, scores, ld, kl,
                            (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_mla_up_project(const void* kv_cache, const void* w_uk, const void* w_uv,
+                                const dsa_kv_desc_t* kv, void* k_nope, void* k_rope, void* v,
+                                int64_t ctx_pad, dsa_stream_t stream) {
+  dsa_q_desc_t qd{kv ? kv->batch : 0, 1, 0, 0};  // keys only: one nominal row per sequence
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, &qd, &g);
+  if (st != DSA_OK) return st;
+  if (!kv_cache || !w_uk || !w_uv || !k_nope || !k_rope || !v) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(kv_cache) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(k_nope) ||
+      !aligned16(k_rope) || !aligned16(v))
+    return DSA_ERR_INVALID_ARG;
+  const MhaPlan m = plan_mha(g);
+  if (ctx_pad < m.ctx_pad || ctx_pad % kMhaTile != 0) return DSA_ERR_INVALID_ARG;
+  if (!mha_fits(g, ctx_pad)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  return launch_up_proj(kv_cache, w_uk, w_uv, g, k_nope, k_rope, v, ctx_pad,
+                        (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_selection_mask(const int32_t* idx, int32_t k, const dsa_kv_desc_t* kv,
+                                const dsa_q_desc_t* qd, uint32_t* mask, int64_t mask_ld,
+                                dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (!idx || !mask || !aligned16(mask)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (mask_ld < plan_mha(g).mask_ld || mask_ld % 4 != 0) return DSA_ERR_INVALID_ARG;
+  return launch_selection_mask(idx, k, g, g.row_begin, g.row_count, mask, mask_ld,
+                               (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_masked_mha(const void* q_mha, const void* k_nope, const void* k_rope,
+                            const void* v, int64_t ctx_pad, const dsa_kv_desc_t* kv,
+                            const dsa_q_desc_t* qd, const uint32_t* mask, int64_t mask_ld,
+                            int32_t k, float scale, void* out, float* lse, dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (!q_mha || !k_nope || !k_rope || !v || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_mha) || !aligned16(k_nope) || !aligned16(k_rope) || !aligned16(v) ||
+      !aligned16(out))
+    return DSA_ERR_INVALID_ARG;
+  const MhaPlan m = plan_mha(g);
+  if (ctx_pad < m.ctx_pad || ctx_pad % kMhaTile != 0) return DSA_ERR_INVALID_ARG;
+  if (!mha_fits(g, ctx_pad)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (mask) {
+    if (!aligned16(mask) || mask_ld < m.mask_ld || mask_ld % 4 != 0) return DSA_ERR_INVALID_ARG;
+    if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (!(scale > 0.f) || !(scale < 1e30f)) return DSA_ERR_INVALID_ARG;
+  return launch_masked_mha(q_mha, k_nope, k_rope, v, ctx_pad, g, mask, mask_ld, mask ? k : 0,
+                           scale, out, lse, (cudaStream_t)stream);
+}
+
+size_t dsa_mha_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k) {
+  Geometry g;
+  if (check_geometry(kv, q, &g) != DSA_OK || k < 1 || k > kMaxK) return 0;
+  const ForwardPlan f = plan_forward(g, k, true);
+  const MhaPlan m = plan_mha(g);
+  return f.idx_bytes + f.score_bytes + m.mask_bytes + m.kn_bytes + m.kr_bytes + m.v_bytes;
+}
+
+dsa_status_t dsa_mha_prefill(const void* q_idx, const float* w, const void* k_idx,
+                             const float* k_scale, const void* q_mha, const void* kv_cache,
+                             const void* w_uk, const void* w_uv, const dsa_kv_desc_t* kv,
+                             const dsa_q_desc_t* qd, int32_t k, float scale, void* workspace,
+                             size_t workspace_bytes, int32_t* idx_out, void* out, float* lse,
+                             dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (!q_idx || !w || !k_idx || !k_scale || !q_mha || !kv_cache || !w_uk || !w_uv || !out ||
+      !lse)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q_mha) || !aligned16(kv_cache) ||
+      !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(out))
+    return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!(scale > 0.f) || !(scale < 1e30f)) return DSA_ERR_INVALID_ARG;
+  ForwardPlan f = plan_forward(g, k, idx_out == nullptr);
+  const MhaPlan m = plan_mha(g);
+  if (!mha_fits(g, m.ctx_pad)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  const size_t fixed = f.idx_bytes + m.mask_bytes + m.kn_bytes + m.kr_bytes + m.v_bytes;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < fixed)
+    return DSA_ERR_WORKSPACE;
+  // Rows that select every visible key (pos + 1 <= k) need no scores. Without a
+  // seqlens array their positions are known here, so the indexer skips them.
+  const int r_end = g.row_begin + g.row_count;
+  int sel_begin = g.row_begin;
+  if (!g.seqlens)
+    sel_begin = std::min(r_end, std::max(g.row_begin, k - g.max_ctx + g.q_per_seq));
+  const int sel_rows = r_end - sel_begin;
+  if (sel_rows > 0) {
+    const int64_t row_bytes = f.ld * 4 * g.batch;
+    int64_t rows = std::min<int64_t>(sel_rows, f.chunk_rows);
+    if ((int64_t)(workspace_bytes - fixed) < rows * row_bytes) {
+      rows = (int64_t)(workspace_bytes - fixed) / row_bytes;
+      if (rows < 1) return DSA_ERR_WORKSPACE;
+      if (rows >= 4) rows &= ~int64_t(3);
+    }
+    f.chunk_rows = (int)rows;
+  }
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws);
+  ws += f.idx_bytes;
+  uint32_t* mask = reinterpret_cast<uint32_t*>(ws);
+  ws += m.mask_bytes;
+  void* k_nope = ws;
+  ws += m.kn_bytes;
+  void* k_rope = ws;
+  ws += m.kr_bytes;
+  void* v = ws;
+  ws += m.v_bytes;
+  float* scores = reinterpret_cast<float*>(ws);
+  cudaStream_t s = (cudaStream_t)stream;
+  // selection for the rows that need it, then their masks
+  if (idx_out && sel_begin > g.row_begin) {  // all-visible rows: no scores are read
+    st = launch_topk(scores, f.ld, g, g.row_begin, sel_begin - g.row_begin, k, idx, s);
+    if (st != DSA_OK) return st;
+  }
+  for (int r0 = sel_begin; r0 < r_end; r0 += f.chunk_rows) {
+    const int rc = std::min(f.chunk_rows, r_end - r0);
+    st = launch_indexer(q_idx, w, k_idx, k_scale, g, scores, f.ld, r0, rc, s);
+    if (st != DSA_OK) return st;
+    st = launch_topk(scores, f.ld, g, r0, rc, k, idx, s);
+    if (st != DSA_OK) return st;
+  }
+  if (sel_rows > 0) {
+    st = launch_selection_mask(idx, k, g, sel_begin, sel_rows, mask, m.mask_ld, s);
+    if (st != DSA_OK) return st;
+  }
+  st = launch_up_proj(kv_cache, w_uk, w_uv, g, k_nope, k_rope, v, m.ctx_pad, s);
+  if (st != DSA_OK) return st;
+  return launch_masked_mha(q_mha, k_nope, k_rope, v, m.ctx_pad, g, sel_rows > 0 ? mask : nullptr,
+                           m.mask_ld, k, scale, out, lse, s);
 }
 
 dsa_status_t dsa_selftest_wait_timeout(dsa_stream_t stream) {

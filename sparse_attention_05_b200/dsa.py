@@ -71,6 +71,18 @@ SIGNATURES = {
     "dsa_forward_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.POINTER(KvDescC),
                                            ctypes.POINTER(QDescC), ctypes.c_int32, ctypes.c_float,
                                            _P, _P, _P, _P]),
+    "dsa_mla_up_project": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(KvDescC), _P, _P, _P,
+                                          ctypes.c_int64, _P]),
+    "dsa_selection_mask": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.POINTER(KvDescC),
+                                          ctypes.POINTER(QDescC), _P, ctypes.c_int64, _P]),
+    "dsa_masked_mha": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int64, ctypes.POINTER(KvDescC),
+                                      ctypes.POINTER(QDescC), _P, ctypes.c_int64, ctypes.c_int32,
+                                      ctypes.c_float, _P, _P, _P]),
+    "dsa_mha_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
+                                                 ctypes.c_int32]),
+    "dsa_mha_prefill": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(KvDescC),
+                                       ctypes.POINTER(QDescC), ctypes.c_int32, ctypes.c_float, _P,
+                                       ctypes.c_size_t, _P, _P, _P, _P]),
     "dsa_get_device_error": (ctypes.c_int, [_P]),
     "dsa_set_wait_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "dsa_selftest_wait_timeout": (ctypes.c_int, [_P]),
@@ -262,6 +274,90 @@ def dsa_forward_noalloc(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_p
                                      _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k,
                                      float(scale), _ptr(idx_out), _ptr(out), _ptr(lse),
                                      _stream(stream)), "dsa_forward_noalloc")
+    return out, lse, idx_out
+
+
+# ---- MLA in MHA mode (masked-MHA emulation of DSA for short prefill) -------------------
+
+MHA_DN, MHA_DR, MHA_DV = 128, 64, 128
+
+
+def mha_ctx_pad(kv: KvLayout) -> int:
+    """Key slots per (sequence, head) of the decompressed keys and values."""
+    return round_up(kv.max_ctx, 128)
+
+
+def dsa_mla_up_project(kv_cache, w_uk, w_uv, kv: KvLayout, k_nope=None, k_rope=None, v=None,
+                       stream=None):
+    """Decompressed MHA-mode keys / values (include/dsa.h): k_nope [B,128,ctx_pad,128],
+    k_rope [B,ctx_pad,64], v [B,128,ctx_pad,128], all bf16."""
+    cp = mha_ctx_pad(kv)
+    dev = kv_cache.device
+    if k_nope is None:
+        k_nope = torch.empty(kv.batch, HEADS, cp, MHA_DN, dtype=torch.bfloat16, device=dev)
+    if k_rope is None:
+        k_rope = torch.empty(kv.batch, cp, MHA_DR, dtype=torch.bfloat16, device=dev)
+    if v is None:
+        v = torch.empty(kv.batch, HEADS, cp, MHA_DV, dtype=torch.bfloat16, device=dev)
+    kvd = kv.c()
+    _check(lib().dsa_mla_up_project(_ptr(kv_cache), _ptr(w_uk), _ptr(w_uv), ctypes.byref(kvd),
+                                    _ptr(k_nope), _ptr(k_rope), _ptr(v), k_nope.shape[2],
+                                    _stream(stream)), "dsa_mla_up_project")
+    return k_nope, k_rope, v
+
+
+def dsa_selection_mask(idx, kv: KvLayout, q_per_seq: int, mask=None, rows=None, stream=None):
+    """Selection bits [T, mask_ld] uint32 (stored as int32) of the window's rows."""
+    T, k = idx.shape
+    if mask is None:
+        mask = torch.zeros(T, mha_ctx_pad(kv) // 32, dtype=torch.int32, device=idx.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    _check(lib().dsa_selection_mask(_ptr(idx), k, ctypes.byref(kvd), ctypes.byref(qd),
+                                    _ptr(mask), mask.shape[1], _stream(stream)),
+           "dsa_selection_mask")
+    return mask
+
+
+def dsa_masked_mha(q_mha, k_nope, k_rope, v, kv: KvLayout, q_per_seq: int, scale: float,
+                   mask=None, k: int = 0, out=None, lse=None, rows=None, stream=None):
+    """Masked MHA (include/dsa.h): out [T,128,128] bf16, lse [T,128] fp32."""
+    T = q_mha.shape[0]
+    if out is None:
+        out = torch.empty(T, HEADS, MHA_DV, dtype=torch.bfloat16, device=q_mha.device)
+    if lse is None:
+        lse = torch.empty(T, HEADS, dtype=torch.float32, device=q_mha.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    _check(lib().dsa_masked_mha(_ptr(q_mha), _ptr(k_nope), _ptr(k_rope), _ptr(v),
+                                k_nope.shape[2], ctypes.byref(kvd), ctypes.byref(qd), _ptr(mask),
+                                mask.shape[1] if mask is not None else 0, int(k), float(scale),
+                                _ptr(out), _ptr(lse), _stream(stream)), "dsa_masked_mha")
+    return out, lse
+
+
+def dsa_mha_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None) -> int:
+    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows)
+    return int(lib().dsa_mha_workspace_size(ctypes.byref(kvd), ctypes.byref(qd), k))
+
+
+def dsa_mha_prefill(q_idx, w, k_idx, k_scale, q_mha, kv_cache, w_uk, w_uv, kv: KvLayout,
+                    q_per_seq: int, k: int, scale: float, workspace=None, idx_out=None,
+                    out=None, lse=None, rows=None, stream=None):
+    """Short-prefill DSA in MHA mode: indexer -> top-k -> masks -> up-projection ->
+    masked MHA, one call (include/dsa.h)."""
+    T = q_mha.shape[0]
+    if workspace is None:
+        nbytes = dsa_mha_workspace_size(kv, T, q_per_seq, k, rows)
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q_mha.device)
+    if out is None:
+        out = torch.empty(T, HEADS, MHA_DV, dtype=torch.bfloat16, device=q_mha.device)
+    if lse is None:
+        lse = torch.empty(T, HEADS, dtype=torch.float32, device=q_mha.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    _check(lib().dsa_mha_prefill(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q_mha),
+                                 _ptr(kv_cache), _ptr(w_uk), _ptr(w_uv), ctypes.byref(kvd),
+                                 ctypes.byref(qd), k, float(scale), _ptr(workspace),
+                                 workspace.numel(), _ptr(idx_out), _ptr(out), _ptr(lse),
+                                 _stream(stream)), "dsa_mha_prefill")
     return out, lse, idx_out
 
 

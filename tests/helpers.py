@@ -73,9 +73,12 @@ def check_index_sets(gpu_idx: np.ndarray, ref_idx: np.ndarray, ref_scores: np.nd
     return n_diff_total
 
 
-def check_attention(o_gpu: np.ndarray, lse_gpu: np.ndarray, o_ref: np.ndarray, lse_ref: np.ndarray):
+def check_attention(o_gpu: np.ndarray, lse_gpu: np.ndarray, o_ref: np.ndarray, lse_ref: np.ndarray,
+                    lse_tol=None, lse_bulk: float = 0.99):
     """bf16 output within OUT_ATOL abs and OUT_RTOL rel (per element, either
-    bound suffices); LSE within LSE_ATOL."""
+    bound suffices); LSE within LSE_ATOL. With ``lse_tol`` (an array shaped like
+    lse_ref) each LSE is held to its own bound instead, and at least ``lse_bulk``
+    of them must still be within LSE_ATOL."""
     o_gpu = o_gpu.astype(np.float64)
     err = np.abs(o_gpu - o_ref)
     bad = (err > OUT_ATOL) & (err > OUT_RTOL * np.abs(o_ref))
@@ -83,5 +86,54 @@ def check_attention(o_gpu: np.ndarray, lse_gpu: np.ndarray, o_ref: np.ndarray, l
     fin = np.isfinite(lse_ref)
     assert np.array_equal(np.isfinite(lse_gpu), fin)
     lerr = np.abs(lse_gpu[fin].astype(np.float64) - lse_ref[fin])
-    assert lerr.max(initial=0.0) <= LSE_ATOL, f"LSE max abs err {lerr.max():.3e}"
+    if lse_tol is None:
+        assert lerr.max(initial=0.0) <= LSE_ATOL, f"LSE max abs err {lerr.max():.3e}"
+    else:
+        over = lerr > np.asarray(lse_tol)[fin]
+        assert not over.any(), f"{over.sum()} LSE values beyond their bound; max err {lerr.max():.3e}"
+        frac = float(np.mean(lerr <= LSE_ATOL)) if lerr.size else 1.0
+        assert frac >= lse_bulk, f"only {frac:.4f} of LSE values within {LSE_ATOL}"
     return float(err.max(initial=0.0)), float(lerr.max(initial=0.0))
+
+
+# fp32 accumulation of the 512-term up-projection dot products: at most 512 additions,
+# each adding one rounding of at most 2^-24 relative (doubled: the tensor core's
+# summation order and internal rounding are not specified)
+UP_PROJ_GAMMA = 2 * 512 * 2.0 ** -24
+
+
+def mha_lse_tolerance(q_mha, kv, q_seq, q_pos, sets, w_uk, scale, rows, *, block_table=None,
+                      page_size=64):
+    """Per (row, head) bound on |LSE_gpu - LSE_oracle| for MHA mode.
+
+    The oracle rounds the exact fp64 keys W^UK c to bf16; the GPU rounds an fp32
+    sum of the same 512 products, which lies within UP_PROJ_GAMMA * sum|c_i w_i|
+    of the exact value, so a key element may land one bf16 step away only where
+    its exact value is that close to a rounding midpoint. Such an element moves
+    logit s by at most scale * |q_d| * (its bf16 step): delta_s. LSE(z + dz) -
+    LSE(z) = ln sum_s p_s e^{dz_s}, so |dLSE| <= ln sum_s p_s e^{delta_s} with the
+    oracle's weights p_s. Adds LSE_ATOL for the remaining fp32 arithmetic."""
+    from oracle import bf16_round, resolve_kv_rows
+    R, H = len(rows), q_mha.shape[1]
+    tol = np.zeros((R, H))
+    d_n = w_uk.shape[1]
+    for b in sorted({int(q_seq[t]) for t in rows}):
+        mine = [r for r, t in enumerate(rows) if int(q_seq[t]) == b]
+        n = max(int(q_pos[rows[r]]) for r in mine) + 1
+        c = np.asarray(resolve_kv_rows(kv, b, list(range(n)), block_table, page_size), np.float64)
+        cl, ca = c[:, :512], np.abs(c[:, :512])
+        for h in range(H):
+            w = np.asarray(w_uk[h], np.float64)
+            k_ex = cl @ w.T
+            eps = UP_PROJ_GAMMA * (ca @ np.abs(w).T)
+            step = np.abs(bf16_round(k_ex + eps).astype(np.float64) -
+                          bf16_round(k_ex - eps).astype(np.float64))
+            k_r = np.concatenate([bf16_round(k_ex).astype(np.float64), c[:, 512:]], axis=1)
+            for r in mine:
+                s = np.asarray(sets[r], np.int64)
+                qv = np.asarray(q_mha[rows[r], h], np.float64)
+                z = scale * (k_r[s] @ qv)
+                pw = np.exp(z - (z.max() + np.log(np.sum(np.exp(z - z.max())))))
+                delta = scale * (step[s] @ np.abs(qv[:d_n]))
+                tol[r, h] = np.log(np.sum(pw * np.exp(delta))) + LSE_ATOL
+    return tol
