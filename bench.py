@@ -47,6 +47,7 @@ WORKLOADS = {
     "prefill_128k": dict(kind="prefill", L=131072, seed=3, n_hot=64),
 }
 DEFAULT_WORKLOAD = "paged_decode_128k"
+MHA_MAX_L = 16384  # MHA mode is the short-prefill path (dense causal cost grows as L^2)
 
 SCORE_BUDGET = 2 << 30  # bytes of fp32 score rows per chunk (as the library's own plan)
 
@@ -99,6 +100,44 @@ def algorithmic_work(p: synth.Problem, k: int = K_SEL) -> dict:
         "indexer_kl": {"bytes": T * (128 * 576 * 2 + 128 * 4 + 4 * k + 4) +
                        (1152 + 4) * int(n_sel.sum()),
                        "flop": 2 * 128 * 576 * int(n_sel.sum()), "flop_dtype": "bf16"},
+    }
+
+
+def algorithmic_work_mha(p: synth.Problem, k: int = K_SEL) -> dict:
+    """Bytes and FLOPs of a short-prefill step in MHA mode, per kernel.
+
+    indexer / top-k: as in MQA mode, for the rows with more than k visible keys
+             (the other rows select every visible key and need no scores).
+    mask:    the selected indices of those rows read, their bit rows written.
+    up-projection: per key the latent row (1152 B) read and 128 heads x (128 key
+             + 128 value) bf16 written, plus both weight tensors once (32 MiB);
+             2 * 512 * 256 * 128 BF16 FLOP per key.
+    masked MHA: Q (128 x 192 bf16), out (128 x 128 bf16) and LSE per row, the
+             decompressed keys/values once, the mask bits; 2 * 128 * (192 + 128)
+             = 81920 BF16 FLOP per visible (row, key) pair: the mode computes the
+             causal triangle and the mask only removes weight.
+    """
+    seqlens = p.seqlens.cpu().long()
+    pos = p.q_pos().long()
+    n_vis = pos + 1
+    sel = n_vis > k
+    T, T_sel = p.num_q, int(sel.sum())
+    keys = int(seqlens.sum())
+    idx_bytes = (132 * keys if T_sel else 0) + T_sel * (64 * 128 * 2 + 64 * 4) + \
+        4 * int(n_vis[sel].sum())
+    return {
+        "indexer": {"bytes": idx_bytes, "flop": 16384 * int(n_vis[sel].sum()),
+                    "flop_dtype": "fp8"},
+        "topk": {"bytes": 4 * int(n_vis[sel].sum()) + 4 * T_sel * k, "flop": 0,
+                 "flop_dtype": None},
+        "mask": {"bytes": 4 * T_sel * k + int(((n_vis[sel] + 127) // 128).sum()) * 16,
+                 "flop": 0, "flop_dtype": None},
+        "up_proj": {"bytes": keys * (1152 + 128 * 256 * 2 + 128) + 2 * 128 * 128 * 512 * 2,
+                    "flop": 2 * 512 * 256 * 128 * keys, "flop_dtype": "bf16"},
+        "masked_mha": {"bytes": T * (128 * 192 * 2 + 128 * 128 * 2 + 128 * 4) +
+                       keys * (128 * 256 * 2 + 128) +
+                       int(((n_vis[sel] + 127) // 128).sum()) * 16,
+                       "flop": 81920 * int(n_vis.sum()), "flop_dtype": "bf16"},
     }
 
 
@@ -261,6 +300,104 @@ class Runner:
             if ev is not None:
                 ev["indexer_kl"].append(_record())
 
+    # end-to-end through the public call dsa_forward
+    def e2e_host_inputs(self):
+        p = self.p
+        h = {"q_idx": p.q_idx, "w": p.w, "q": p.q, "seqlens": p.seqlens}
+        if p.paged:
+            h["block_table"] = p.block_table
+        return h
+
+    def e2e_workspace(self):
+        d, p = self.dsa, self.p
+        return max(256, d.dsa_workspace_size(self.kv, p.num_q, p.q_per_seq, self.k))
+
+    def e2e_call(self, g, kv, ws, out, lse, stream):
+        d, p = self.dsa, self.p
+        d.dsa_forward(g["q_idx"], g["w"], p.k_idx, p.k_scale, g["q"], p.kv, kv, p.q_per_seq,
+                      self.k, p.scale, workspace=ws, out=out, lse=lse, stream=stream)
+
+
+class MhaRunner:
+    """Short-prefill step in MHA mode through the library's stage calls (the same
+    launches dsa_mha_prefill makes): indexer + top-k for the rows with more than
+    k visible keys, their selection masks, the up-projection of the latent cache
+    and the masked MHA."""
+
+    STAGES = ("indexer", "topk", "mask", "up_proj", "masked_mha")
+
+    def __init__(self, p: synth.Problem, k: int = K_SEL, seed: int = 0):
+        from sparse_attention_05_b200 import dsa
+        if p.q_per_seq != p.max_ctx:
+            raise SystemExit("--mode mha runs the prefill workloads")
+        self.dsa, self.p, self.k = dsa, p, k
+        self.m = synth.mha_inputs(p, seed + 500, device=p.q.device)
+        self.kv = dsa.KvLayout.of(p)
+        T, B, dev = p.num_q, p.batch, p.q.device
+        self.ld = dsa.round_up(p.max_ctx, 128)
+        sel_begin = min(p.q_per_seq, max(0, k))   # row i selects all of 0..i when i < k
+        n_sel = p.q_per_seq - sel_begin
+        rows = max(1, SCORE_BUDGET // (self.ld * 4 * B))
+        if rows >= n_sel:
+            rows = max(1, n_sel)
+        elif rows >= 4:
+            rows &= ~3
+        self.sel = (sel_begin, n_sel)
+        self.chunks = [(r0, min(rows, p.q_per_seq - r0)) for r0 in range(sel_begin, p.q_per_seq, rows)]
+        self.scores = torch.empty(B * rows, self.ld, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        cp = dsa.mha_ctx_pad(self.kv)
+        self.mask = torch.zeros(T, cp // 32, dtype=torch.int32, device=dev)
+        self.kn = torch.empty(B, 128, cp, 128, dtype=torch.bfloat16, device=dev)
+        self.kr = torch.empty(B, cp, 64, dtype=torch.bfloat16, device=dev)
+        self.vv = torch.empty(B, 128, cp, 128, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(T, 128, 128, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(T, 128, dtype=torch.float32, device=dev)
+        self.launches_per_step = 2 * len(self.chunks) + (1 if n_sel else 0) + 2
+
+    def step(self, ev=None):
+        d, p, m = self.dsa, self.p, self.m
+
+        def mark(name):
+            if ev is not None:
+                ev[name].append(_record())
+        for r0, rc in self.chunks:
+            mark("indexer")
+            d.dsa_indexer_scores(p.q_idx, p.w, p.k_idx, p.k_scale, self.kv, p.q_per_seq,
+                                 scores=self.scores[: p.batch * rc], rows=(r0, rc))
+            mark("indexer")
+            mark("topk")
+            d.dsa_topk(self.scores[: p.batch * rc], self.kv, p.q_per_seq, self.k, idx=self.idx,
+                       rows=(r0, rc))
+            mark("topk")
+        if self.sel[1]:
+            mark("mask")
+            d.dsa_selection_mask(self.idx, self.kv, p.q_per_seq, mask=self.mask, rows=self.sel)
+            mark("mask")
+        mark("up_proj")
+        d.dsa_mla_up_project(p.kv, m.w_uk, m.w_uv, self.kv, self.kn, self.kr, self.vv)
+        mark("up_proj")
+        mark("masked_mha")
+        d.dsa_masked_mha(m.q_mha, self.kn, self.kr, self.vv, self.kv, p.q_per_seq, p.scale,
+                         mask=self.mask if self.sel[1] else None, k=self.k, out=self.out,
+                         lse=self.lse)
+        mark("masked_mha")
+
+    # end-to-end through the public composed call
+    def e2e_host_inputs(self):
+        return {"q_idx": self.p.q_idx, "w": self.p.w, "q_mha": self.m.q_mha,
+                "seqlens": self.p.seqlens}
+
+    def e2e_workspace(self):
+        d, p = self.dsa, self.p
+        return max(256, d.dsa_mha_workspace_size(self.kv, p.num_q, p.q_per_seq, self.k))
+
+    def e2e_call(self, g, kv, ws, out, lse, stream):
+        d, p, m = self.dsa, self.p, self.m
+        d.dsa_mha_prefill(g["q_idx"], g["w"], p.k_idx, p.k_scale, g["q_mha"], p.kv, m.w_uk,
+                          m.w_uv, kv, p.q_per_seq, self.k, p.scale, workspace=ws, out=out,
+                          lse=lse, stream=stream)
+
 
 def _record():
     e = torch.cuda.Event(enable_timing=True)
@@ -308,9 +445,10 @@ def job_throughput(world: int, rows_per_rank: int, steps: int, max_secs: float) 
     return world * rows_per_rank * steps / max_secs
 
 
-def e2e_run(r: Runner, steps: int, warmup: int, world: int):
-    """Through the public call dsa_forward, with the step's query-side inputs
-    copied from pinned host memory and the result read back every step.
+def e2e_run(r, steps: int, warmup: int, world: int):
+    """Through the public call (dsa_forward; dsa_mha_prefill in MHA mode), with
+    the step's query-side inputs copied from pinned host memory and the result
+    read back every step.
 
     Copies and compute overlap across steps the way a serving loop would run
     them: step i's inputs go up on an upload stream while step i-1 computes,
@@ -318,15 +456,12 @@ def e2e_run(r: Runner, steps: int, warmup: int, world: int):
     computes (two device buffers for each). Every step still makes its own
     full host->device and device->host copies inside the timed region."""
     d, p = r.dsa, r.p
-    host = {n: getattr(p, n).cpu().pin_memory() for n in ("q_idx", "w", "q", "seqlens")}
-    if p.paged:
-        host["block_table"] = p.block_table.cpu().pin_memory()
+    host = {n: v.cpu().pin_memory() for n, v in r.e2e_host_inputs().items()}
     dev = [{n: torch.empty_like(v, device="cuda") for n, v in host.items()} for _ in range(2)]
     outs = [(torch.empty_like(r.out), torch.empty_like(r.lse)) for _ in range(2)]
     outs_h = [(torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory(),
                torch.empty(r.lse.shape, dtype=r.lse.dtype).pin_memory()) for _ in range(2)]
-    ws = torch.empty(max(256, d.dsa_workspace_size(r.kv, p.num_q, p.q_per_seq, r.k)),
-                     dtype=torch.uint8, device="cuda")
+    ws = torch.empty(r.e2e_workspace(), dtype=torch.uint8, device="cuda")
     kvs = [d.KvLayout(batch=p.batch, max_ctx=p.max_ctx, seqlens=dev[b]["seqlens"],
                       block_table=dev[b].get("block_table"), page_size=p.page_size,
                       num_pages=r.kv.num_pages) for b in range(2)]
@@ -346,10 +481,7 @@ def e2e_run(r: Runner, steps: int, warmup: int, world: int):
             s_cmp.wait_event(ev["in_ready"][b])
             if i >= 2:
                 s_cmp.wait_event(ev["out_free"][b])
-            g = dev[b]
-            d.dsa_forward(g["q_idx"], g["w"], p.k_idx, p.k_scale, g["q"], p.kv, kvs[b],
-                          p.q_per_seq, r.k, p.scale, workspace=ws, out=outs[b][0],
-                          lse=outs[b][1], stream=s_cmp)
+            r.e2e_call(dev[b], kvs[b], ws, outs[b][0], outs[b][1], s_cmp)
             ev["in_free"][b].record(s_cmp)
             ev["done"][b].record(s_cmp)
         with torch.cuda.stream(s_down):
@@ -419,6 +551,25 @@ def oracle_step(inp, scale, k=K_SEL):
                           ld=inp["ld"])
 
 
+def oracle_step_mha(p: synth.Problem, m: synth.MhaInputs, rows, k=K_SEL):
+    """The oracle's MHA-mode prefill for ``rows``: indexer + top-k for the rows with
+    more than k visible keys, then the masked MHA (every visible key otherwise)."""
+    from oracle import indexer_scores, masked_mha, topk_rows
+    inp = oracle_sample_inputs(p, rows)
+    trows = torch.as_tensor(list(rows))
+    q_mha = m.q_mha[trows].float().cpu().numpy()
+    local = np.arange(len(rows))
+    need = [r for r in local if inp["q_pos"][r] + 1 > k]
+    idx = [np.arange(int(inp["q_pos"][r]) + 1) for r in local]
+    if need:
+        sc = indexer_scores(inp["q_idx"], inp["w"], inp["k_idx"], inp["k_scale"], inp["q_seq"],
+                            inp["q_pos"], ld=inp["ld"], rows=need)
+        for r, sel in zip(need, topk_rows(sc, inp["q_pos"], k, rows=need)):
+            idx[r] = sel
+    return masked_mha(q_mha, inp["kv"], inp["q_seq"], inp["q_pos"], idx, p.scale,
+                      m.w_uk.float().cpu().numpy(), m.w_uv.float().cpu().numpy())
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -428,22 +579,33 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(p: synth.Problem, name: str, budget_s: float = 12.0, seed: int = 0) -> dict:
+def cpu_baseline(p: synth.Problem, name: str, budget_s: float = 12.0, seed: int = 0,
+                 mha=None) -> dict:
+    """The oracle on a bounded sample: two query rows of a random sequence per call
+    (their last rows in MQA mode; two random rows in MHA mode, whose cost is the
+    up-projection of every visible key per head), until ``budget_s`` of host time."""
     rng = np.random.default_rng(seed)
     rows_done, elapsed, seqs = 0, 0.0, []
     while elapsed < budget_s and rows_done < p.num_q:
         b = int(rng.integers(0, p.batch))
         r0 = b * p.q_per_seq
-        rows = list(range(r0, r0 + min(p.q_per_seq, 2)))
-        inp = oracle_sample_inputs(p, rows)
-        t0 = time.perf_counter()
-        oracle_step(inp, p.scale)
+        if mha is None:
+            rows = list(range(r0, r0 + min(p.q_per_seq, 2)))
+            inp = oracle_sample_inputs(p, rows)
+            t0 = time.perf_counter()
+            oracle_step(inp, p.scale)
+        else:
+            rows = sorted(r0 + int(i) for i in rng.choice(p.q_per_seq, 2, replace=False))
+            t0 = time.perf_counter()
+            oracle_step_mha(p, mha, rows)
         elapsed += time.perf_counter() - t0
         rows_done += len(rows)
         seqs.append(b)
+    what = ("indexer+top-k (rows past k)+masked MHA per row" if mha is not None
+            else "full indexer+top-k+attention per row")
     return {"value": rows_done / elapsed, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"{rows_done} query rows of {name} (sequences {seqs[:8]}"
-                      f"{'...' if len(seqs) > 8 else ''}), full indexer+top-k+attention per row, "
+                      f"{'...' if len(seqs) > 8 else ''}), {what}, "
                       f"{elapsed:.1f} s of host time"}
 
 
@@ -456,9 +618,16 @@ def reference_arm(args):
     p = make_problem(args.workload, dev)
     rng = np.random.default_rng(123)
     per_step_rows = min(p.q_per_seq, 2)
+    m = synth.mha_inputs(p, 500, device=dev) if args.mode == "mha" else None
 
     def one():
         b = int(rng.integers(0, p.batch))
+        if m is not None:
+            rows = sorted(b * p.q_per_seq + int(i)
+                          for i in rng.choice(p.q_per_seq, per_step_rows, replace=False))
+            t0 = time.perf_counter()
+            oracle_step_mha(p, m, rows)
+            return time.perf_counter() - t0
         rows = list(range(b * p.q_per_seq, b * p.q_per_seq + per_step_rows))
         inp = oracle_sample_inputs(p, rows)
         t0 = time.perf_counter()
@@ -474,6 +643,7 @@ def reference_arm(args):
             "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, **WORKLOADS[args.workload],
+                       **({"mode": "mha (masked MHA emulation of DSA)"} if m is not None else {}),
                        "sample_rows_per_step": per_step_rows},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
                              "kind": "oracle",
@@ -499,18 +669,31 @@ def main(argv=None):
                     help="also run the indexer KL loss term (training target) every step")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the decode batch (small cases for profiler captures)")
+    ap.add_argument("--mode", default="mqa", choices=["mqa", "mha"],
+                    help="mha: short-prefill DSA in MLA's MHA mode (masked MHA; prefill_8k)")
     ap.add_argument("--soak-s", type=float, default=1.0,
                     help="untimed seconds of steps right before the timed region (clock samples)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
 
+    if args.mode == "mha":
+        w = WORKLOADS[args.workload]
+        if w["kind"] != "prefill" or w["L"] > MHA_MAX_L:
+            raise SystemExit(f"--mode mha is the short-prefill path: prefill workloads with "
+                             f"L <= {MHA_MAX_L} (not {args.workload})")
+        if args.kl:
+            raise SystemExit("--kl runs with the MQA-mode path")
     if args.impl == "reference":
         return reference_arm(args)
 
     world, rank, local = dist_setup(args.gpus)
     p = make_problem(args.workload, "cuda", seed_offset=rank, batch=args.batch)
-    r = Runner(p, with_kl=args.kl)
-    work = algorithmic_work(p)
+    if args.mode == "mha":
+        r = MhaRunner(p, seed=rank)
+        work = algorithmic_work_mha(p)
+    else:
+        r = Runner(p, with_kl=args.kl)
+        work = algorithmic_work(p)
     peaks = load_peaks()
 
     for _ in range(args.warmup):
@@ -523,7 +706,10 @@ def main(argv=None):
         torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    ev = {"indexer": [], "topk": [], "sparse_mla": []}
+    if args.mode == "mha":
+        ev = {n: [] for n in MhaRunner.STAGES}
+    else:
+        ev = {"indexer": [], "topk": [], "sparse_mla": []}
     if args.kl:
         ev["indexer_kl"] = []
     start = _record()
@@ -536,7 +722,7 @@ def main(argv=None):
     secs_local = start.elapsed_time(stop) / 1e3
     secs = max_over_ranks(secs_local, world)
 
-    per_kernel = {kname: _pairs_ms(e) for kname, e in ev.items()}
+    per_kernel = {kname: _pairs_ms(e) for kname, e in ev.items() if e}
     launches = {kname: len(v) for kname, v in per_kernel.items()}
     total_ms = {kname: sum(v) for kname, v in per_kernel.items()}
     dominant = max(total_ms, key=total_ms.get)
@@ -557,13 +743,16 @@ def main(argv=None):
     e2e = None if args.no_e2e else e2e_run(r, max(3, args.steps // 2), 3, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(p, args.workload)
+        cpu = cpu_baseline(p, args.workload, mha=r.m if args.mode == "mha" else None)
 
     if rank == 0:
         cfg = {"workload": args.workload, **WORKLOADS[args.workload],
                **({"batch": args.batch} if args.batch else {}),
                **({"indexer_kl": True} if args.kl else {}), "k": K_SEL,
-               "heads": 128, "d_qk": 576, "d_v": 512, "h_idx": 64, "d_idx": 128,
+               **({"mode": "mha (masked MHA emulation of DSA)", "heads": 128, "d_qk": 192,
+                   "d_v": 128, "d_latent": 576} if args.mode == "mha" else
+                  {"heads": 128, "d_qk": 576, "d_v": 512}),
+               "h_idx": 64, "d_idx": 128,
                "query_rows_per_gpu": p.num_q,
                "l2": "inputs larger than L2 (no flush)",
                "parallelism": f"dp{world} (independent sequences per GPU)"}

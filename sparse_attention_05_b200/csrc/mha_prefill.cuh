@@ -373,10 +373,13 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // heaviest row blocks (most key tiles) first
-  const int64_t per_rb = (int64_t)p.batch * kMhaHeads;
-  const int rb = p.row_blocks - 1 - (int)(blockIdx.x / per_rb);
-  const int64_t bh = blockIdx.x % per_rb;
+  // Head-major order: the CTAs resident together are the row blocks of one or two
+  // (sequence, head) pairs, which read the same key/value tiles, so each tile comes
+  // from HBM about once and from L2 after that (all heads of one row block at once
+  // would stream every tile from HBM once per row block). Within a head the
+  // heaviest row blocks (most key tiles) go first.
+  const int64_t bh = blockIdx.x / p.row_blocks;
+  const int rb = p.row_blocks - 1 - (int)(blockIdx.x % p.row_blocks);
   const int b = (int)(bh / kMhaHeads), h = (int)(bh % kMhaHeads);
   const int i0 = rb * kMhaTile;  // first window row of the block
   const int seqlen = mha_seqlen(p.seqlens, b, p.max_ctx);
@@ -540,19 +543,26 @@ __global__ void __launch_bounds__(kFaThreads, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32u(tmem_base + st * kMhaTile + c * 32 + lane_off, x[c]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_wait_ld_fence(x[c]);
-      // logits in base 2; keys outside the row's set are -inf
-      float mt = -INFINITY;
+      // Keys outside the row's set become -inf. One 32-bit validity word per
+      // 32-key chunk (causal limit AND selection bits); the running max of the raw
+      // scores uses four independent accumulators (a single warp per SM
+      // sub-partition runs each row, so dependent chains, not issue, set its pace).
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const uint32_t bits = c == 0 ? mw.x : c == 1 ? mw.y : c == 2 ? mw.z : mw.w;
+        const int lim = pos - kbase - 32 * c;  // last visible key of the chunk
+        const uint32_t vm =
+            bits & (lim >= 31 ? 0xffffffffu : (lim < 0 ? 0u : (2u << lim) - 1u));
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const bool vis = (kbase + 32 * c + e <= pos) && ((bits >> e) & 1u);
-          const float z = vis ? __uint_as_float(x[c][e]) * p.scale_log2 : -INFINITY;
-          x[c][e] = __float_as_uint(z);
-          mt = fmaxf(mt, z);
+          const float v = ((vm >> e) & 1u) ? __uint_as_float(x[c][e]) : -INFINITY;
+          x[c][e] = __float_as_uint(v);
+          mx[e & 3] = fmaxf(mx[e & 3], v);
         }
       }
+      // tile max in base-2 logits (the scale is positive)
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
       // lazy rescale: the reference max moves only when it grows by more than 8
       const bool grow = m_ref != -INFINITY && mt > m_ref + 8.f;
       if (__any_sync(0xffffffffu, grow)) {
@@ -581,20 +591,24 @@ __global__ void __launch_bounds__(kFaThreads, 1)
       if (m_ref == -INFINITY) m_ref = mt;  // first visible key (stays -inf without one)
       // P = 2^(z - m_ref), rounded to bf16 for the MMA, written over the first 64
       // columns of the scores
-      const float mref = m_ref == -INFINITY ? 0.f : m_ref;
+      // p = 2^(s * scale_log2 - m_ref) as one FFMA and one ex2 per key (-inf -> 0)
+      const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
+      const float s2 = p.scale_log2;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         float pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int c = (64 * h2 + 2 * e) >> 5, w = (64 * h2 + 2 * e) & 31;
-          const float p0 = ex2_approx(__uint_as_float(x[c][w]) - mref);
-          const float p1 = ex2_approx(__uint_as_float(x[c][w + 1]) - mref);
-          l += p0 + p1;  // the softmax sum from the unrounded values (exact LSE)
+          const float p0 = ex2_approx(fmaf(__uint_as_float(x[c][w]), s2, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(x[c][w + 1]), s2, neg_m));
+          ls[e & 3] += p0 + p1;  // the softmax sum from the unrounded values (exact LSE)
           pk[e] = __uint_as_float(pack_bf16x2(p0, p1));
         }
         tmem_st32(tmem_base + st * kMhaTile + h2 * 32 + lane_off, pk);
       }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&pfull[st]));
