@@ -177,7 +177,7 @@ def roofline(kernel: str, work: dict, avg_s: float, peaks: dict, long_step: bool
 
 def dram_traffic(kernel: str, workload: str):
     """Per-launch DRAM bytes from a committed ncu summary, if it matches the
-    kernel source that is built now (else null)."""
+    kernel's source as built now (its header and the PTX helpers; else null)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
@@ -187,7 +187,7 @@ def dram_traffic(kernel: str, workload: str):
         if not e:
             return None
         from sparse_attention_05_b200.build import source_digest
-        if e.get("source_digest") != source_digest():
+        if e.get("source_digest") != source_digest(kernel):
             return None
         return e["bytes_per_launch"]
     except Exception:

@@ -31,13 +31,22 @@ def _nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def source_digest() -> str:
-    """Digest of the CUDA sources and the ABI header (identifies a kernel build)."""
+# the header that holds each kernel (for per-kernel digests)
+KERNEL_HEADER = {"indexer": "indexer.cuh", "topk": "topk.cuh", "sparse_mla": "sparse_mla.cuh",
+                 "indexer_kl": "indexer_kl.cuh", "mask": "mha_prefill.cuh",
+                 "up_proj": "mha_prefill.cuh", "masked_mha": "mha_prefill.cuh"}
+
+
+def source_digest(kernel=None) -> str:
+    """Digest of the CUDA sources and the ABI header (identifies a library build);
+    with ``kernel``, of that kernel's header and the shared PTX helpers only."""
     import hashlib
     h = hashlib.sha256()
-    for f in SOURCES + HEADERS:
+    files = (["ptx.cuh", KERNEL_HEADER[kernel]] if kernel else SOURCES + HEADERS)
+    for f in files:
         h.update(open(os.path.join(CSRC, f), "rb").read())
-    h.update(open(os.path.join(ROOT, "include", "dsa.h"), "rb").read())
+    if not kernel:
+        h.update(open(os.path.join(ROOT, "include", "dsa.h"), "rb").read())
     return h.hexdigest()[:16]
 
 
