@@ -169,8 +169,6 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   p.G = std::min(4, row_count);
   p.groups_per_seq = (row_count + p.G - 1) / p.G;
   p.num_groups = g.batch * p.groups_per_seq;
-  p.scale_bulk = (reinterpret_cast<uintptr_t>(k_scale) % 16 == 0) &&
-                 (p.paged ? g.page_size % 64 == 0 : g.max_ctx % 4 == 0);
   p.timeout_ns = g_timeout_ns.load();
   // every CTA takes an equal share of all key tiles (at most one CTA per tile)
   const int64_t max_tiles = (int64_t)p.num_groups * ((g.max_ctx + kIdxTile - 1) / kIdxTile);

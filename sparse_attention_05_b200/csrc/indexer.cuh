@@ -20,16 +20,16 @@
 //
 // Warp roles (384 threads):
 //   warp 0      producer: TMA key tiles (2 boxes of 64 rows x 128 B, 128-B swizzle)
-//               issued by lane 0, and the tile's 128 key scales staged by the
-//               whole warp with cp.async into a ring beside the key stages
+//               issued by lane 0, page lookups batched by the warp
 //   warp 1      TMEM allocation + single-thread tcgen05.mma issue
 //   warps 2-3   query quantizers: bf16 -> E4M3 rows in the canonical swizzled
 //               K-major layout, w*s_q per row (double-buffered per unit)
 //   warps 4-11  epilogue: two warpgroups; tiles alternate between them and
 //               cycle through 512 / N TMEM accumulators (2 to 8), so the MMA
-//               can run that many tiles ahead; thread = key lane
-// A stage of the ring is reused only after the MMA has read its keys and the
-// epilogue has read its scales.
+//               can run that many tiles ahead; thread = key lane, which loads
+//               its key's scale from global memory itself, one tile ahead
+// A stage of the ring carries key codes only and is reused as soon as the MMA has
+// read it (the scales never gate a stage).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -47,8 +47,7 @@ constexpr int kIdxStageBytes = kIdxTile * kIdxDim;  // 16 KB of e4m3
 constexpr int kIdxQBufBytes = 4 * kIdxHeads * kIdxDim;  // G <= 4 rows x 64 heads x 128 B
 constexpr int kIdxSmemBytes =
     1024 /*align slack*/ + kIdxStages * kIdxStageBytes + 2 * kIdxQBufBytes +
-    2 * 4 * kIdxHeads * 4 /*wq*/ + kIdxStages * kIdxTile * 4 /*key scales*/ +
-    512 /*barriers etc*/ + 512 /*share + scan scratch*/;
+    2 * 4 * kIdxHeads * 4 /*wq*/ + 512 /*barriers etc*/ + 512 /*share + scan scratch*/;
 constexpr int kIdxMaxAcc = 8;  // TMEM accumulators: 512 / N, at most 8
 
 struct IndexerParams {
@@ -65,7 +64,6 @@ struct IndexerParams {
   int32_t G;                     // query rows per MMA (N = 64 G)
   int32_t groups_per_seq;        // ceil(row_count / G)
   int32_t num_groups;            // batch * groups_per_seq
-  int32_t scale_bulk;            // k_scale rows keep 16-B alignment for 4-key pieces
   uint64_t timeout_ns;
 };
 
@@ -193,8 +191,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint8_t* stages = smem;
   uint8_t* qbuf = stages + kIdxStages * kIdxStageBytes;
   float* wq = reinterpret_cast<float*>(qbuf + 2 * kIdxQBufBytes);  // [2][256]
-  float* sscale = wq + 2 * 4 * kIdxHeads;                              // [stages][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sscale + kIdxStages * kIdxTile);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wq + 2 * 4 * kIdxHeads);
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + kIdxStages;
   uint64_t* tfull = bars + 2 * kIdxStages;
@@ -217,8 +214,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kIdxStages; ++s) {
-      mbar_init(smem_u32(&kfull[s]), 1 + 32);    // expect_tx arrival + 32 scale copiers
-      mbar_init(smem_u32(&kempty[s]), 1 + 128);  // MMA commit + the epilogue warpgroup
+      mbar_init(smem_u32(&kfull[s]), 1);   // expect_tx arrival (+ the tile's bytes)
+      mbar_init(smem_u32(&kempty[s]), 1);  // the MMA's commit
     }
     for (int i = 0; i < kIdxMaxAcc; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);
@@ -303,23 +300,6 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             tma_load_2d(smem_u32(stages + st * kIdxStageBytes + h * 8192), &tm_keys, bar, 0,
                         (int)base[h]);
         }
-        // key scales: lane l copies keys 4l .. 4l+3 of the tile, as one 16-B
-        // piece (zero-filled past the last visible key) when the cache rows
-        // keep 16-B alignment, else as four 4-B pieces
-        {
-          const int h = lane >> 4, e = lane * 4;
-          const int nvis = live[h] ? min(4, max(0, pos_max + 1 - (kt * kIdxTile + e))) : 0;
-          const float* src = p.k_scale + (nvis > 0 ? base[h] + (e & 63) : 0);
-          if (p.scale_bulk) {
-            cp_async_16(smem_u32(sscale + st * kIdxTile + e), src, 4u * (uint32_t)nvis);
-          } else {
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              cp_async_4(smem_u32(sscale + st * kIdxTile + e + v), src + (v < nvis ? v : 0),
-                         v < nvis ? 4u : 0u);
-          }
-        }
-        cp_async_mbar_arrive(bar);
       }
       if (!ok) break;
     }
@@ -327,7 +307,6 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     if (lane == 0)
       for (uint32_t j = it > kIdxStages ? it - kIdxStages : 0; j < it; ++j)
         mbar_wait(smem_u32(&kfull[j % kIdxStages]), (j / kIdxStages) & 1, TO, no_abort);
-    cp_async_wait_all();
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -450,17 +429,31 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       if (!warp_wait(smem_u32(&qfull[qb]), (un >> 1) & 1, TO, abort_flag)) break;
       const float* wrow = wq + qb * 4 * kIdxHeads;
       const int pos0 = U.seqlen - p.q_per_seq + U.i0;  // position of the group's first row
+      const int pos_max = pos0 + U.nrows - 1;
+      // this thread's key scale of tile kt (0 past the last visible key or behind
+      // an invalid page entry, whose scores are masked or reported anyway)
+      auto scale_of = [&](int kt) -> float {
+        const int s = kt * kIdxTile + e;
+        if (s > pos_max) return 0.f;
+        int64_t row = (int64_t)U.b * p.max_ctx + s;
+        if (p.paged) {
+          const int pg = __ldg(p.block_table + (int64_t)U.b * p.max_pages + s / p.page_size);
+          if (pg < 0 || pg >= p.num_pages) return 0.f;
+          row = (int64_t)pg * p.page_size + s % p.page_size;
+        }
+        return __ldg(p.k_scale + row);
+      };
+      int pf_kt = -1;  // the tile whose scale is already in flight (this warpgroup's next)
+      float pf_ks = 0.f;
       bool ok = true;
       for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
         if ((int)(it & 1) != wg) continue;  // the other warpgroup's tile
-        const int st = it % kIdxStages;
         const int s = kt * kIdxTile + e;
-        if (!warp_wait(smem_u32(&kfull[st]), (it / kIdxStages) & 1, TO, abort_flag)) {
-          ok = false;
-          break;
+        const float ks = pf_kt == kt ? pf_ks : scale_of(kt);
+        if (kt + 2 < U.kt1) {
+          pf_ks = scale_of(kt + 2);
+          pf_kt = kt + 2;
         }
-        const float ks = sscale[st * kIdxTile + e];
-        mbar_arrive(smem_u32(&kempty[st]));
         const int ab = (int)(it % (uint32_t)nacc);  // accumulator of this tile
         if (!warp_wait(smem_u32(&tfull[ab]), (it / nacc) & 1, TO, abort_flag)) {
           ok = false;
