@@ -110,12 +110,13 @@ __device__ __forceinline__ bool idx_next(const IndexerParams& p, const IdxShare&
   return false;
 }
 
-// Work is balanced on a cost of (tiles + kIdxUnitCost) per group: a group's
-// query rows are quantized once per unit, which is worth about 16 tiles, so
-// many short causal groups (early prefill rows) weigh what they cost. A cost
-// position x within a group maps to the tile boundary max(0, x - kIdxUnitCost);
-// neighbouring shares apply the same map to their common boundary.
-constexpr int kIdxUnitCost = 16;
+// Work is balanced on a cost of (tiles + G * kIdxRowCost) per group: a group's G
+// query rows are quantized once per unit (64 rows of 128 elements each), which
+// is worth about 8 tiles per row, so many short causal groups (early prefill
+// rows) weigh what they cost. A cost position x within a group maps to the tile
+// boundary max(0, x - unit cost); neighbouring shares apply the same map to
+// their common boundary.
+constexpr int kIdxRowCost = 8;
 
 // Block-wide: the exact share [W c / n, W (c+1) / n) of the total cost W.
 __device__ void idx_share(const IndexerParams& p, IdxShare* out, uint32_t* scratch) {
@@ -142,10 +143,11 @@ __device__ void idx_share(const IndexerParams& p, IdxShare* out, uint32_t* scrat
     excl = before + incl - v;
     total = all;
   };
+  const long long unit_cost = (long long)kIdxRowCost * p.G;
   auto cost_of = [&](int grp, int& nt) -> long long {
     IdxUnit U;
     nt = grp < p.num_groups ? idx_group(p, grp, U) : 0;
-    return nt > 0 ? (long long)nt + kIdxUnitCost : 0;
+    return nt > 0 ? (long long)nt + unit_cost : 0;
   };
   // pass 1: total cost
   long long W = 0;
@@ -171,11 +173,11 @@ __device__ void idx_share(const IndexerParams& p, IdxShare* out, uint32_t* scrat
     const long long a = run + excl, e = a + cost;  // cost positions [a, e) belong to grp
     if (cost > 0 && a <= lo && lo < e) {
       out->gs = grp;
-      out->ts = (int)max(0ll, lo - a - kIdxUnitCost);
+      out->ts = (int)max(0ll, lo - a - unit_cost);
     }
     if (cost > 0 && a < hi && hi <= e) {
       out->ge = grp;
-      out->te = (int)max(0ll, hi - a - kIdxUnitCost);
+      out->te = (int)max(0ll, hi - a - unit_cost);
     }
     run += tot;
   }
