@@ -70,7 +70,7 @@ def make_problem(name: str, device, seed_offset: int = 0, batch=None) -> synth.P
     return synth.prefill(device=device, **w)
 
 
-def algorithmic_work(p: synth.Problem, k: int = K_SEL) -> dict:
+def algorithmic_work(p: synth.Problem, k: int = K_SEL, rows=None) -> dict:
     """Bytes and FLOPs the method must move or compute per step, per kernel.
 
     indexer: 132 B per visible key per sequence (128 B E4M3 + 4 B scale), the
@@ -82,9 +82,11 @@ def algorithmic_work(p: synth.Problem, k: int = K_SEL) -> dict:
     """
     seqlens = p.seqlens.cpu().long()
     pos = p.q_pos().long()
+    if rows is not None:  # a subset of the query rows (context-parallel ranks)
+        pos = pos[torch.as_tensor(rows)]
     n_vis = pos + 1
     n_sel = torch.clamp(n_vis, max=k)
-    T = p.num_q
+    T = len(pos)
     keys = int(seqlens.sum())  # every sequence's keys are read once
     idx_bytes = 132 * keys + T * (64 * 128 * 2 + 64 * 4) + 4 * int(n_vis.sum())
     idx_flop = 16384 * int(n_vis.sum())
@@ -316,6 +318,58 @@ class Runner:
         d, p = self.dsa, self.p
         d.dsa_forward(g["q_idx"], g["w"], p.k_idx, p.k_scale, g["q"], p.kv, kv, p.q_per_seq,
                       self.k, p.scale, workspace=ws, out=out, lse=lse, stream=stream)
+
+
+class CpRunner(Runner):
+    """Context-parallel prefill on this rank: the rank owns a contiguous token shard
+    of the per-token caches; every step all-gathers them (NCCL) and runs the stage
+    calls on the rank's zigzag query rows (row windows of the library calls)."""
+
+    def __init__(self, p: synth.Problem, world: int, rank: int, k: int = K_SEL):
+        from sparse_attention_05_b200 import cp
+        super().__init__(p, k)
+        self.cp, self.world = cp, world
+        L = p.max_ctx
+        b, e = cp.token_shard(L, world, rank)
+        self.shards = {n: getattr(p, n)[0, b:e].clone() for n in ("k_idx", "k_scale", "kv")}
+        self.windows = cp.zigzag_windows(L, world, rank)
+        self.rows = [i for r0, rc in self.windows for i in range(r0, r0 + rc)]
+        # score chunks inside each window (the same budget as the single-GPU plan)
+        per = max(1, SCORE_BUDGET // (self.ld * 4 * p.batch))
+        if per >= 4:
+            per &= ~3
+        self.chunks = [(r0 + c, min(per, rc - c)) for r0, rc in self.windows
+                       for c in range(0, rc, per)]
+        self.launches_per_step = 2 * len(self.chunks) + len(self.windows)
+
+    def step(self, ev=None):
+        d, p = self.dsa, self.p
+        if ev is not None:
+            ev["allgather"].append(_record())
+        full = {n: self.cp.allgather_cache(t, p.max_ctx, self.world)
+                for n, t in self.shards.items()}
+        k_idx, k_scale, kv = full["k_idx"][None], full["k_scale"][None], full["kv"][None]
+        if ev is not None:
+            ev["allgather"].append(_record())
+        for r0, rc in self.chunks:
+            if ev is not None:
+                ev["indexer"].append(_record())
+            d.dsa_indexer_scores(p.q_idx, p.w, k_idx, k_scale, self.kv, p.q_per_seq,
+                                 scores=self.scores[: p.batch * rc], rows=(r0, rc))
+            if ev is not None:
+                ev["indexer"].append(_record())
+                ev["topk"].append(_record())
+            d.dsa_topk(self.scores[: p.batch * rc], self.kv, p.q_per_seq, self.k, idx=self.idx,
+                       rows=(r0, rc))
+            if ev is not None:
+                ev["topk"].append(_record())
+        for r0, rc in self.windows:
+            if ev is not None:
+                ev["sparse_mla"].append(_record())
+            d.dsa_sparse_mla_fwd(p.q, kv, self.kv, p.q_per_seq, self.idx, p.scale, out=self.out,
+                                 lse=self.lse, rows=(r0, rc))
+            if ev is not None:
+                ev["sparse_mla"].append(_record())
 
 
 class MhaRunner:
@@ -669,6 +723,9 @@ def main(argv=None):
                     help="also run the indexer KL loss term (training target) every step")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the decode batch (small cases for profiler captures)")
+    ap.add_argument("--cp", action="store_true",
+                    help="context-parallel prefill: caches sharded by token, all-gathered "
+                         "every step, query rows split zigzag across the ranks")
     ap.add_argument("--mode", default="mqa", choices=["mqa", "mha"],
                     help="mha: short-prefill DSA in MLA's MHA mode (masked MHA; prefill_8k)")
     ap.add_argument("--soak-s", type=float, default=1.0,
@@ -686,9 +743,20 @@ def main(argv=None):
     if args.impl == "reference":
         return reference_arm(args)
 
+    if args.cp and (WORKLOADS[args.workload]["kind"] != "prefill" or args.mode != "mqa"
+                    or args.kl):
+        raise SystemExit("--cp runs the prefill workloads in MQA mode")
     world, rank, local = dist_setup(args.gpus)
-    p = make_problem(args.workload, "cuda", seed_offset=rank, batch=args.batch)
-    if args.mode == "mha":
+    # context parallel: one sequence shared by all ranks (same seed everywhere)
+    p = make_problem(args.workload, "cuda", seed_offset=0 if args.cp else rank,
+                     batch=args.batch)
+    if args.cp:
+        r = CpRunner(p, world, rank)
+        work = algorithmic_work(p, rows=r.rows)
+        L = p.max_ctx
+        work["allgather"] = {"bytes": L * (128 + 4 + 1152) * (world - 1) // max(world, 1),
+                             "flop": 0, "flop_dtype": None}
+    elif args.mode == "mha":
         r = MhaRunner(p, seed=rank)
         work = algorithmic_work_mha(p)
     else:
@@ -708,6 +776,8 @@ def main(argv=None):
     torch.cuda.synchronize()
     if args.mode == "mha":
         ev = {n: [] for n in MhaRunner.STAGES}
+    elif args.cp:
+        ev = {"allgather": [], "indexer": [], "topk": [], "sparse_mla": []}
     else:
         ev = {"indexer": [], "topk": [], "sparse_mla": []}
     if args.kl:
@@ -725,7 +795,8 @@ def main(argv=None):
     per_kernel = {kname: _pairs_ms(e) for kname, e in ev.items() if e}
     launches = {kname: len(v) for kname, v in per_kernel.items()}
     total_ms = {kname: sum(v) for kname, v in per_kernel.items()}
-    dominant = max(total_ms, key=total_ms.get)
+    # the dominant kernel (the all-gather of the context-parallel mode is a collective)
+    dominant = max((k for k in total_ms if k != "allgather"), key=total_ms.get)
     long_step = secs / args.steps > 0.05
     avg_s = total_ms[dominant] / 1e3 / args.steps  # one step's worth of that kernel
     roof = roofline(dominant, work, avg_s, peaks, long_step)
@@ -740,7 +811,8 @@ def main(argv=None):
                          "bound": rf["bound"], "frac": rf["frac"],
                          "achieved": rf["achieved"], "unit": rf["unit"]}
 
-    e2e = None if args.no_e2e else e2e_run(r, max(3, args.steps // 2), 3, world)
+    # context parallel: the end-to-end arm of the public call is the single-GPU one
+    e2e = None if (args.no_e2e or args.cp) else e2e_run(r, max(3, args.steps // 2), 3, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(p, args.workload, mha=r.m if args.mode == "mha" else None)
@@ -753,14 +825,19 @@ def main(argv=None):
                    "d_v": 128, "d_latent": 576} if args.mode == "mha" else
                   {"heads": 128, "d_qk": 576, "d_v": 512}),
                "h_idx": 64, "d_idx": 128,
-               "query_rows_per_gpu": p.num_q,
+               "query_rows_per_gpu": len(r.rows) if args.cp else p.num_q,
                "l2": "inputs larger than L2 (no flush)",
-               "parallelism": f"dp{world} (independent sequences per GPU)"}
+               "parallelism": (f"cp{world} (caches sharded by token and all-gathered every "
+                               f"step, query rows zigzag across GPUs)" if args.cp else
+                               f"dp{world} (independent sequences per GPU)")}
+        # context parallel: the job processes one sequence's L rows per step
+        rows_job = p.num_q if args.cp else world * p.num_q
         line = {
-            "metric": METRIC, "value": job_throughput(world, p.num_q, args.steps, secs),
+            "metric": METRIC, "value": rows_job * args.steps / secs,
             "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+            "scaling": "strong" if args.cp else "weak",
             "vs_baseline": None, "dtype": "e4m3+bf16", "data": "synthetic", "config": cfg,
             "roofline": roof, "stages": stages, "clocks": clk,
             "gpu_launches": sum(launches.values()),
