@@ -264,3 +264,34 @@ def test_host_argument_checks():
     with pytest.raises(dsa.DSAError) as e:
         dsa.dsa_selection_mask(idx, kv, 256, mask=bad)
     assert e.value.status == 1
+
+
+# ---- degenerate cases ------------------------------------------------------------------
+
+
+def test_one_token_sequences_attend_to_themselves():
+    """Sequences of one token: the row's only key is itself, so o = v and LSE = z
+    (the oracle's closed form for one key)."""
+    p = synth.decode(batch=3, ctx=1, q_per_seq=1, seed=105)
+    m = synth.mha_inputs(p, 106)
+    o_g, l_g, _ = _gpu_mha(p, m)
+    _check(p, m, o_g, l_g, None, np.arange(p.num_q))
+
+
+def test_k_one_every_row_selects_a_single_key():
+    p = synth.prefill(L=300, seed=107)
+    m = synth.mha_inputs(p, 108)
+    idx = _random_idx(p, 1, 109)
+    o_g, l_g, _ = _gpu_mha(p, m, idx=idx, k=1)
+    rows = np.arange(0, 300, 7)
+    _check(p, m, o_g[rows], l_g[rows], idx[rows], rows)
+
+
+def test_paged_cache_with_selection_masks():
+    p = synth.paged_decode(batch=2, q_per_seq=160, min_ctx=400, max_ctx=640, page_size=64,
+                           seed=111)
+    m = synth.mha_inputs(p, 112)
+    idx = _random_idx(p, 200, 113)
+    o_g, l_g, _ = _gpu_mha(p, m, idx=idx, k=200)
+    rows = synth.sample_rows(p.num_q, 30, seed=114, must=(0, 159, 160, 319)).numpy()
+    _check(p, m, o_g[rows], l_g[rows], idx[rows], rows)
