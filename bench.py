@@ -372,6 +372,35 @@ class CpRunner(Runner):
                 ev["sparse_mla"].append(_record())
 
 
+class FusedRunner(Runner):
+    """The fused indexer -> top-k selection (no stored score rows; one host sync per
+    chunk of rows inside the call) followed by the sparse MLA."""
+
+    def __init__(self, p: synth.Problem, k: int = K_SEL):
+        super().__init__(p, k)
+        d = self.dsa
+        nbytes = d.dsa_fused_workspace_size(self.kv, p.num_q, p.q_per_seq, k)
+        self.ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=p.q.device)
+        self.scores = None  # never materialised
+        # per chunk: sampled indexer, threshold top-k, filtering indexer, selection
+        per = max(1, (2 << 30) // (p.batch * (self.ld // 8 * 4 + 12 + 8192 * 8)))
+        self.launches_per_step = 4 * (-(-p.q_per_seq // per)) + 1
+
+    def step(self, ev=None):
+        d, p = self.dsa, self.p
+        if ev is not None:
+            ev["select_fused"].append(_record())
+        d.dsa_select_fused(p.q_idx, p.w, p.k_idx, p.k_scale, self.kv, p.q_per_seq, self.k,
+                           idx=self.idx, workspace=self.ws)
+        if ev is not None:
+            ev["select_fused"].append(_record())
+            ev["sparse_mla"].append(_record())
+        d.dsa_sparse_mla_fwd(p.q, p.kv, self.kv, p.q_per_seq, self.idx, p.scale, out=self.out,
+                             lse=self.lse)
+        if ev is not None:
+            ev["sparse_mla"].append(_record())
+
+
 class MhaRunner:
     """Short-prefill step in MHA mode through the library's stage calls (the same
     launches dsa_mha_prefill makes): indexer + top-k for the rows with more than
@@ -726,6 +755,8 @@ def main(argv=None):
     ap.add_argument("--cp", action="store_true",
                     help="context-parallel prefill: caches sharded by token, all-gathered "
                          "every step, query rows split zigzag across the ranks")
+    ap.add_argument("--fused", action="store_true",
+                    help="fused indexer -> top-k selection (no stored score rows)")
     ap.add_argument("--mode", default="mqa", choices=["mqa", "mha"],
                     help="mha: short-prefill DSA in MLA's MHA mode (masked MHA; prefill_8k)")
     ap.add_argument("--soak-s", type=float, default=1.0,
@@ -750,7 +781,14 @@ def main(argv=None):
     # context parallel: one sequence shared by all ranks (same seed everywhere)
     p = make_problem(args.workload, "cuda", seed_offset=0 if args.cp else rank,
                      batch=args.batch)
-    if args.cp:
+    if args.fused and (args.cp or args.mode != "mqa" or args.kl):
+        raise SystemExit("--fused runs the MQA-mode path alone")
+    if args.fused:
+        r = FusedRunner(p)
+        work = algorithmic_work(p)
+        # the fused selection does the indexer's work (plus a 1/8 sample) and the top-k's
+        work["select_fused"] = dict(work["indexer"])
+    elif args.cp:
         r = CpRunner(p, world, rank)
         work = algorithmic_work(p, rows=r.rows)
         L = p.max_ctx
@@ -778,6 +816,8 @@ def main(argv=None):
         ev = {n: [] for n in MhaRunner.STAGES}
     elif args.cp:
         ev = {"allgather": [], "indexer": [], "topk": [], "sparse_mla": []}
+    elif args.fused:
+        ev = {"select_fused": [], "sparse_mla": []}
     else:
         ev = {"indexer": [], "topk": [], "sparse_mla": []}
     if args.kl:
@@ -812,7 +852,8 @@ def main(argv=None):
                          "achieved": rf["achieved"], "unit": rf["unit"]}
 
     # context parallel: the end-to-end arm of the public call is the single-GPU one
-    e2e = None if (args.no_e2e or args.cp) else e2e_run(r, max(3, args.steps // 2), 3, world)
+    e2e = None if (args.no_e2e or args.cp or args.fused) else \
+        e2e_run(r, max(3, args.steps // 2), 3, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(p, args.workload, mha=r.m if args.mode == "mha" else None)
@@ -820,7 +861,8 @@ def main(argv=None):
     if rank == 0:
         cfg = {"workload": args.workload, **WORKLOADS[args.workload],
                **({"batch": args.batch} if args.batch else {}),
-               **({"indexer_kl": True} if args.kl else {}), "k": K_SEL,
+               **({"indexer_kl": True} if args.kl else {}),
+               **({"selection": "fused indexer -> top-k"} if args.fused else {}), "k": K_SEL,
                **({"mode": "mha (masked MHA emulation of DSA)", "heads": 128, "d_qk": 192,
                    "d_v": 128, "d_latent": 576} if args.mode == "mha" else
                   {"heads": 128, "d_qk": 576, "d_v": 512}),
@@ -840,7 +882,9 @@ def main(argv=None):
             "scaling": "strong" if args.cp else "weak",
             "vs_baseline": None, "dtype": "e4m3+bf16", "data": "synthetic", "config": cfg,
             "roofline": roof, "stages": stages, "clocks": clk,
-            "gpu_launches": sum(launches.values()),
+            # our kernels launched in the timed region (the fused selection's event
+            # pair spans its four launches per chunk of rows)
+            "gpu_launches": r.launches_per_step * args.steps,
             "e2e": e2e, "cpu_baseline": cpu, "peaks": peaks,
         }
         print(json.dumps(line))

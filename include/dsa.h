@@ -200,6 +200,46 @@ DSA_API dsa_status_t dsa_forward_noalloc(const void* q_idx, const float* w, cons
                                          int32_t* idx_out, void* out, float* lse,
                                          dsa_stream_t stream);
 
+/* ---- Fused indexer -> top-k: the selection without stored score rows ------------------
+ * The same selection as dsa_indexer_scores + dsa_topk (report §1 and §2.1: S_t =
+ * Top-k(I_{t,:}); equal scores keep the lower position, ascending, -1 padded),
+ * without ever writing a row's scores to memory:
+ *   1. a strided pass scores every 8th 128-key tile of each row and takes the m-th
+ *      largest of that sample as the row's threshold (m = k/8 + 6 sqrt(k/8) + 32,
+ *      so the threshold lies well below the row's k-th score);
+ *   2. a second pass scores every key and keeps, per row, the keys at or above the
+ *      threshold as candidates (at most cand_cap per row);
+ *   3. the exact top-k of the candidates is selected. A row whose candidates are
+ *      fewer than k or more than cand_cap cannot be decided from them; such rows
+ *      (rare) are selected from their full score rows, so the result is always
+ *      identical to dsa_indexer_scores + dsa_topk.
+ * The call synchronizes `stream` once per chunk of rows to read the count of such
+ * rows. Requires max_ctx <= 131072.
+ *  cand_cap  candidates kept per row, 0 = 8192 (the most); smaller values force the
+ *            full-row path more often (a test hook)
+ *  workspace 256-byte aligned, dsa_fused_workspace_size() bytes for the largest chunk
+ *            of rows; smaller workspaces (down to one row per sequence) take smaller
+ *            chunks
+ *  idx       int32 [T][k] out, as dsa_topk writes it. */
+DSA_API size_t dsa_fused_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q,
+                                        int32_t k);
+DSA_API dsa_status_t dsa_select_fused(const void* q_idx, const float* w, const void* k_idx,
+                                      const float* k_scale, const dsa_kv_desc_t* kv,
+                                      const dsa_q_desc_t* qd, int32_t k, int32_t cand_cap,
+                                      void* workspace, size_t workspace_bytes, int32_t* idx,
+                                      dsa_stream_t stream);
+
+/* dsa_forward with the fused selection: dsa_select_fused then dsa_sparse_mla_fwd.
+ * Arguments as dsa_forward plus cand_cap; the workspace holds the indices (unless
+ * idx_out is given) followed by dsa_select_fused's workspace. */
+DSA_API dsa_status_t dsa_forward_fused(const void* q_idx, const float* w, const void* k_idx,
+                                       const float* k_scale, const void* q,
+                                       const void* kv_cache, const dsa_kv_desc_t* kv,
+                                       const dsa_q_desc_t* qd, int32_t k, float scale,
+                                       int32_t cand_cap, void* workspace, size_t workspace_bytes,
+                                       int32_t* idx_out, void* out, float* lse,
+                                       dsa_stream_t stream);
+
 /* ---- MLA in MHA mode: the masked-MHA emulation of DSA for short prefill ----------
  * Report Appendix A (Fig. 4): MLA runs in an MHA mode (training, prefill) or an MQA
  * mode (decode); report §3 "Inference cost": for short-sequence prefill a masked MHA

@@ -8,7 +8,9 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <cmath>
 #include <mutex>
+#include <vector>
 
 #include "../../include/dsa.h"
 #include "ptx.cuh"
@@ -89,7 +91,8 @@ int num_sms() {
 
 // ---- top-k launch ------------------------------------------------------------------
 dsa_status_t launch_topk(const float* scores, int64_t ld, const Geometry& g, int row_begin,
-                         int row_count, int k, int32_t* idx, cudaStream_t stream) {
+                         int row_count, int k, int32_t* idx, cudaStream_t stream,
+                         int tile_stride = 1, float* kth_out = nullptr) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -97,7 +100,8 @@ dsa_status_t launch_topk(const float* scores, int64_t ld, const Geometry& g, int
                                     kTopkSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
-  TopkParams p{scores, ld, g.seqlens, g.max_ctx, g.q_per_seq, row_begin, row_count, g.batch, k, idx};
+  TopkParams p{scores, ld, g.seqlens, g.max_ctx, g.q_per_seq, row_begin, row_count, g.batch, k,
+               idx, tile_stride, kth_out};
   const int64_t grid = (int64_t)g.batch * row_count;
   if (grid == 0) return DSA_OK;
   topk_kernel<<<(unsigned)grid, kTopkThreads, kTopkSmemBytes, stream>>>(p);
@@ -135,9 +139,19 @@ dsa_status_t make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType
 }
 
 // ---- indexer launch -----------------------------------------------------------------
+// Candidate output of the indexer's filter mode (see IndexerParams).
+struct IdxFilter {
+  const float* thr = nullptr;
+  uint32_t* cand_key = nullptr;
+  int32_t* cand_pos = nullptr;
+  uint32_t* cand_cnt = nullptr;
+  int cand_cap = 0;
+};
+
 dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx,
                             const float* k_scale, const Geometry& g, float* scores, int64_t ld,
-                            int row_begin, int row_count, cudaStream_t stream) {
+                            int row_begin, int row_count, cudaStream_t stream,
+                            int tile_stride = 1, const IdxFilter& filt = IdxFilter()) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -169,6 +183,12 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   p.G = std::min(4, row_count);
   p.groups_per_seq = (row_count + p.G - 1) / p.G;
   p.num_groups = g.batch * p.groups_per_seq;
+  p.tile_stride = tile_stride;
+  p.thr = filt.thr;
+  p.cand_key = filt.cand_key;
+  p.cand_pos = filt.cand_pos;
+  p.cand_cnt = filt.cand_cnt;
+  p.cand_cap = filt.cand_cap;
   p.timeout_ns = g_timeout_ns.load();
   // every CTA takes an equal share of all key tiles (at most one CTA per tile)
   const int64_t max_tiles = (int64_t)p.num_groups * ((g.max_ctx + kIdxTile - 1) / kIdxTile);
@@ -448,6 +468,117 @@ dsa_status_t launch_masked_mha(const void* q_mha, const void* k_nope, const void
   return cuda_status(cudaGetLastError());
 }
 
+// ---- fused indexer -> top-k (score rows never stored) ------------------------------------
+constexpr int kFuseStride = 8;  // the threshold pass scores every 8th key tile
+
+dsa_status_t launch_cand_select(const Geometry& g, int row_begin, int row_count, int k,
+                                int32_t* idx, const uint32_t* ckey, const int32_t* cpos,
+                                const uint32_t* cnt, int cap, int32_t* redo_rows,
+                                uint32_t* redo_cnt, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(cand_select_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kCandSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  CandParams p{ckey, cpos, cnt, cap, g.seqlens, g.max_ctx, g.q_per_seq, row_begin, row_count,
+               g.batch, k, idx, redo_rows, redo_cnt};
+  const int64_t grid = (int64_t)g.batch * row_count;
+  if (grid == 0) return DSA_OK;
+  cand_select_kernel<<<(unsigned)grid, kCandThreads, kCandSmemBytes, stream>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+struct FusedPlan {
+  int64_t ld;           // full score row stride (fallback rows)
+  int64_t ld_s;         // sampled score row stride
+  int cap;              // candidates kept per row
+  int m;                // rank of the threshold within a row's sample
+  int chunk_rows;       // window rows per sequence per chunk
+  size_t idx_bytes, fallback_bytes, row_bytes;  // row_bytes: per window row of a chunk
+};
+
+FusedPlan plan_fused(const Geometry& g, int k, bool need_idx, int cap) {
+  FusedPlan f;
+  f.ld = (int64_t)(g.max_ctx + kIdxTile - 1) / kIdxTile * kIdxTile;
+  const int64_t tiles = f.ld / kIdxTile;
+  f.ld_s = ((tiles + kFuseStride - 1) / kFuseStride) * kIdxTile;
+  f.cap = cap > 0 ? cap : kCandCap;
+  // the k / S largest of a row's sample are expected above its k-th score; the
+  // threshold sits 6 standard deviations (and 32) lower, so about 8 (k/S + ...)
+  // keys pass per row and fewer than k only far out in the tail (those rows, and
+  // rows with more than `cap`, take the full path)
+  const int ks = (k + kFuseStride - 1) / kFuseStride;
+  f.m = ks + 6 * (int)std::ceil(std::sqrt((double)ks)) + 32;
+  f.idx_bytes = need_idx ? align256((size_t)g.num_q * k * 4) : 0;
+  f.fallback_bytes = align256((size_t)g.batch * f.ld * 4);
+  f.row_bytes = (size_t)f.ld_s * 4 + 4 /*thr*/ + 4 /*cnt*/ + (size_t)f.cap * 8 + 4 /*redo*/;
+  int64_t rows = std::max<int64_t>(1, kScoreBudgetBytes / ((int64_t)f.row_bytes * g.batch));
+  f.chunk_rows = (int)std::min<int64_t>(rows, g.row_count);
+  if (f.chunk_rows >= 4 && f.chunk_rows < g.row_count) f.chunk_rows &= ~3;
+  return f;
+}
+
+// One chunk of window rows through the fused path; `ws` holds the chunk's buffers.
+dsa_status_t select_fused_chunk(const void* q_idx, const float* w, const void* k_idx,
+                                const float* k_scale, const Geometry& g, const FusedPlan& f,
+                                int k, int r0, int rc, uint8_t* ws, float* fb_scores,
+                                int32_t* idx, cudaStream_t s) {
+  const int64_t nrow = (int64_t)g.batch * rc;
+  float* samp = reinterpret_cast<float*>(ws);
+  ws += align256((size_t)nrow * f.ld_s * 4);
+  float* thr = reinterpret_cast<float*>(ws);
+  ws += align256((size_t)nrow * 4);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ws);
+  ws += align256((size_t)nrow * 4 + 4);  // + the redo counter
+  uint32_t* redo_cnt = cnt + nrow;
+  int32_t* redo_rows = reinterpret_cast<int32_t*>(ws);
+  ws += align256((size_t)nrow * 4);
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(ws);
+  ws += align256((size_t)nrow * f.cap * 4);
+  int32_t* cpos = reinterpret_cast<int32_t*>(ws);
+  if (cudaMemsetAsync(cnt, 0, (size_t)(nrow + 1) * 4, s) != cudaSuccess) return DSA_ERR_CUDA;
+  // 1. thresholds: the m-th largest score of a strided sample of each row's keys
+  dsa_status_t st = launch_indexer(q_idx, w, k_idx, k_scale, g, samp, f.ld_s, r0, rc, s,
+                                   kFuseStride);
+  if (st == DSA_OK) st = launch_topk(samp, f.ld_s, g, r0, rc, f.m, nullptr, s, kFuseStride, thr);
+  // 2. all keys again, keeping only those at or above the row's threshold
+  IdxFilter filt;
+  filt.thr = thr;
+  filt.cand_key = ckey;
+  filt.cand_pos = cpos;
+  filt.cand_cnt = cnt;
+  filt.cand_cap = f.cap;
+  if (st == DSA_OK) st = launch_indexer(q_idx, w, k_idx, k_scale, g, samp, f.ld_s, r0, rc, s, 1, filt);
+  // 3. the exact top-k of each row's candidates
+  if (st == DSA_OK)
+    st = launch_cand_select(g, r0, rc, k, idx, ckey, cpos, cnt, f.cap, redo_rows, redo_cnt, s);
+  if (st != DSA_OK) return st;
+  // 4. rows whose candidates cannot be exact (fewer than k, or more than the list
+  //    holds) are selected from their full score rows
+  uint32_t n_redo = 0;
+  if (cudaMemcpyAsync(&n_redo, redo_cnt, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (n_redo == 0) return DSA_OK;
+  n_redo = std::min<uint32_t>(n_redo, (uint32_t)nrow);
+  std::vector<int32_t> rows(n_redo);
+  if (cudaMemcpy(rows.data(), redo_rows, (size_t)n_redo * 4, cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  std::vector<char> done(rc, 0);  // a window row index covers that row of every sequence
+  for (int32_t wr : rows) {
+    const int ii = wr % rc;
+    if (done[ii]) continue;
+    done[ii] = 1;
+    st = launch_indexer(q_idx, w, k_idx, k_scale, g, fb_scores, f.ld, r0 + ii, 1, s);
+    if (st == DSA_OK) st = launch_topk(fb_scores, f.ld, g, r0 + ii, 1, k, idx, s);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
 // ---- scratch for the allocation-free forward ------------------------------------------
 // A fixed device array that every device loading this library holds until exit.
 // Host code must not use the symbol's host-side address: the device address is
@@ -724,6 +855,73 @@ dsa_status_t dsa_mha_prefill(const void* q_idx, const float* w, const void* k_id
   if (st != DSA_OK) return st;
   return launch_masked_mha(q_mha, k_nope, k_rope, v, m.ctx_pad, g, sel_rows > 0 ? mask : nullptr,
                            m.mask_ld, k, scale, out, lse, s);
+}
+
+size_t dsa_fused_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k) {
+  Geometry g;
+  if (check_geometry(kv, q, &g) != DSA_OK || k < 1 || k > kMaxK) return 0;
+  const FusedPlan f = plan_fused(g, k, true, 0);
+  return f.idx_bytes + f.fallback_bytes +
+         (size_t)f.chunk_rows * g.batch * f.row_bytes + 8 * 256;
+}
+
+dsa_status_t dsa_select_fused(const void* q_idx, const float* w, const void* k_idx,
+                              const float* k_scale, const dsa_kv_desc_t* kv,
+                              const dsa_q_desc_t* qd, int32_t k, int32_t cand_cap,
+                              void* workspace, size_t workspace_bytes, int32_t* idx,
+                              dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (!q_idx || !w || !k_idx || !k_scale || !idx) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (cand_cap < 0 || cand_cap > kCandCap) return DSA_ERR_INVALID_ARG;
+  if ((g.max_ctx + 31) / 32 > kCandMaxWords) return DSA_ERR_UNSUPPORTED_SHAPE;
+  FusedPlan f = plan_fused(g, k, false, cand_cap);
+  const size_t fixed = f.fallback_bytes + 8 * 256;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < fixed)
+    return DSA_ERR_WORKSPACE;
+  const int64_t fit = (int64_t)(workspace_bytes - fixed) / ((int64_t)f.row_bytes * g.batch);
+  if (fit < 1) return DSA_ERR_WORKSPACE;
+  f.chunk_rows = (int)std::min<int64_t>(fit, g.row_count);
+  if (f.chunk_rows >= 4 && f.chunk_rows < g.row_count) f.chunk_rows &= ~3;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  float* fb_scores = reinterpret_cast<float*>(ws);
+  ws += f.fallback_bytes;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int r_end = g.row_begin + g.row_count;
+  for (int r0 = g.row_begin; r0 < r_end; r0 += f.chunk_rows) {
+    const int rc = std::min(f.chunk_rows, r_end - r0);
+    st = select_fused_chunk(q_idx, w, k_idx, k_scale, g, f, k, r0, rc, ws, fb_scores, idx, s);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
+dsa_status_t dsa_forward_fused(const void* q_idx, const float* w, const void* k_idx,
+                               const float* k_scale, const void* q, const void* kv_cache,
+                               const dsa_kv_desc_t* kv, const dsa_q_desc_t* qd, int32_t k,
+                               float scale, int32_t cand_cap, void* workspace,
+                               size_t workspace_bytes, int32_t* idx_out, void* out, float* lse,
+                               dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !kv_cache || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!(scale > 0.f) || !(scale < 1e30f)) return DSA_ERR_INVALID_ARG;
+  const size_t idx_bytes = idx_out ? 0 : align256((size_t)g.num_q * k * 4);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < idx_bytes)
+    return DSA_ERR_WORKSPACE;
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(workspace);
+  st = dsa_select_fused(q_idx, w, k_idx, k_scale, kv, qd, k, cand_cap,
+                        reinterpret_cast<uint8_t*>(workspace) + idx_bytes,
+                        workspace_bytes - idx_bytes, idx, stream);
+  if (st != DSA_OK) return st;
+  return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, (cudaStream_t)stream);
 }
 
 dsa_status_t dsa_selftest_wait_timeout(dsa_stream_t stream) {

@@ -64,6 +64,18 @@ struct IndexerParams {
   int32_t G;                     // query rows per MMA (N = 64 G)
   int32_t groups_per_seq;        // ceil(row_count / G)
   int32_t num_groups;            // batch * groups_per_seq
+  // Strided sample: only key tiles 0, S, 2S, ... of each row (S = tile_stride >= 1);
+  // sample tile u is stored at score columns [128 u, 128 u + 128).
+  int32_t tile_stride;
+  // Filter mode (thr != nullptr): instead of storing scores, the keys of window row
+  // r whose score is >= thr[r] are appended to the row's candidate list as
+  // (order-preserving key, position); cand_cnt[r] counts them (and may exceed
+  // cand_cap, in which case the list holds an arbitrary cand_cap of them).
+  const float* thr;
+  uint32_t* cand_key;            // [batch * row_count][cand_cap]
+  int32_t* cand_pos;             // [batch * row_count][cand_cap]
+  uint32_t* cand_cnt;            // [batch * row_count], zeroed by the caller
+  int32_t cand_cap;
   uint64_t timeout_ns;
 };
 
@@ -81,7 +93,7 @@ __device__ __forceinline__ int idx_group(const IndexerParams& p, int grp, IdxUni
   U.i0 = p.row_begin + g * p.G;
   U.nrows = min(p.G, p.row_begin + p.row_count - U.i0);
   const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
-  return pos_max / kIdxTile + 1;
+  return (pos_max / kIdxTile) / p.tile_stride + 1;  // tiles 0, S, ..., up to pos_max's
 }
 
 // This CTA's share of the tile list: from (group gs, tile ts) to the exclusive
@@ -258,7 +270,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       // for a batch of 16 tiles starting at kb, and the next batch is already
       // in flight, so no tile waits on a block-table load.
       auto fetch_pages = [&](int kb) -> int {
-        const int kt = kb + (lane >> 1), s0 = kt * kIdxTile + (lane & 1) * 64;
+        const int kt = kb + (lane >> 1), s0 = kt * p.tile_stride * kIdxTile + (lane & 1) * 64;
         if (!p.paged || kt >= U.kt1 || s0 > pos_max) return -1;
         return __ldg(p.block_table + (int64_t)U.b * p.max_pages + s0 / p.page_size);
       };
@@ -277,19 +289,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
         const uint32_t bar = smem_u32(&kfull[st]);
         // cache rows of the tile's two 64-key halves (a half never straddles a page)
-        int64_t base[2] = {0, 0};
-        bool live[2] = {false, false};
+        int64_t base[2] = {0, 0};  // half tiles past pos_max or behind a bad page load row 0
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int s0 = kt * kIdxTile + h * 64;
+          const int s0 = kt * p.tile_stride * kIdxTile + h * 64;
           const int page = __shfl_sync(0xffffffffu, pg_cur, 2 * (kt - kb) + h);
           if (s0 <= pos_max) {
             if (!p.paged) {
               base[h] = (int64_t)U.b * p.max_ctx + s0;
-              live[h] = true;
             } else if (page >= 0 && page < p.num_pages) {
               base[h] = (int64_t)page * p.page_size + s0 % p.page_size;
-              live[h] = true;
             } else if (lane == 0) {
               report_error(kErrBounds);
             }
@@ -432,10 +441,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       const float* wrow = wq + qb * 4 * kIdxHeads;
       const int pos0 = U.seqlen - p.q_per_seq + U.i0;  // position of the group's first row
       const int pos_max = pos0 + U.nrows - 1;
+      float thr_row[4] = {0.f, 0.f, 0.f, 0.f};  // filter mode: the rows' thresholds
+      if (p.thr)
+        for (int gi = 0; gi < U.nrows; ++gi)
+          thr_row[gi] = __ldg(p.thr + (int64_t)U.b * p.row_count + (U.i0 - p.row_begin) + gi);
       // this thread's key scale of tile kt (0 past the last visible key or behind
       // an invalid page entry, whose scores are masked or reported anyway)
-      auto scale_of = [&](int kt) -> float {
-        const int s = kt * kIdxTile + e;
+      auto scale_of = [&](int kt) -> float {  // kt: the unit's tile index (strided)
+        const int s = kt * p.tile_stride * kIdxTile + e;
         if (s > pos_max) return 0.f;
         int64_t row = (int64_t)U.b * p.max_ctx + s;
         if (p.paged) {
@@ -450,7 +463,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       bool ok = true;
       for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
         if ((int)(it & 1) != wg) continue;  // the other warpgroup's tile
-        const int s = kt * kIdxTile + e;
+        const int s = kt * p.tile_stride * kIdxTile + e;  // this thread's key
         const float ks = pf_kt == kt ? pf_ks : scale_of(kt);
         if (kt + 2 < U.kt1) {
           pf_ks = scale_of(kt + 2);
@@ -492,7 +505,22 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           const float acc = (a0 + a1) + (a2 + a3);
           const float out = (s <= pos0 + gi) ? ks * acc : -INFINITY;
           const int64_t orow = (int64_t)U.b * p.row_count + (U.i0 - p.row_begin) + gi;
-          p.scores[orow * p.ld + s] = out;
+          if (!p.thr) {
+            p.scores[orow * p.ld + kt * kIdxTile + e] = out;
+          } else {  // filter mode: append (key, position) when the score reaches thr
+            const bool take = s <= pos0 + gi && out >= thr_row[gi];
+            const uint32_t ballot = __ballot_sync(0xffffffffu, take);
+            if (ballot) {
+              uint32_t base = 0;
+              if (lane == __ffs(ballot) - 1) base = atomicAdd(p.cand_cnt + orow, __popc(ballot));
+              base = __shfl_sync(0xffffffffu, base, __ffs(ballot) - 1);
+              const uint32_t slot = base + __popc(ballot & ((1u << lane) - 1u));
+              if (take && slot < (uint32_t)p.cand_cap) {
+                p.cand_key[orow * p.cand_cap + slot] = score_key(out);
+                p.cand_pos[orow * p.cand_cap + slot] = s;
+              }
+            }
+          }
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&tempty[ab]));

@@ -42,8 +42,18 @@ struct TopkParams {
   int32_t row_count;
   int32_t batch;
   int32_t k;
-  int32_t* idx;           // [batch * q_per_seq][k]
+  int32_t* idx;           // [batch * q_per_seq][k], or nullptr: no index output
+  // Sampled rows (tile_stride S > 1): a row holds only key tiles 0, S, 2S, ... of the
+  // visible keys, compacted; its length is (pos / 128 / S + 1) * 128 (the tail of
+  // the last tile is -inf where it lies past pos).
+  int32_t tile_stride;
+  float* kth_out;         // [batch * row_count] or nullptr: the k-th largest score
 };
+
+// Inverse of score_key (a key back to its fp32 value; +0.0 for a zero).
+__device__ __forceinline__ float key_score(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
 
 // fp32 -> key with the same order (as values); -0.0 maps to +0.0.
 __device__ __forceinline__ uint32_t score_key(float x) {
@@ -194,18 +204,23 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
   const int i = p.row_begin + blockIdx.x % p.row_count;
   const int64_t t = (int64_t)b * p.q_per_seq + i;
   const int tid = threadIdx.x;
-  int32_t* out = p.idx + t * p.k;
+  int32_t* out = p.idx ? p.idx + t * p.k : nullptr;
 
   const int seqlen = p.seqlens ? p.seqlens[b] : p.max_ctx;
   if (seqlen < p.q_per_seq || seqlen > p.max_ctx) {
     if (tid == 0) report_error(kErrBounds);
-    for (int j = tid; j < p.k; j += kTopkThreads) out[j] = -1;
+    if (out)
+      for (int j = tid; j < p.k; j += kTopkThreads) out[j] = -1;
+    if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = -INFINITY;
     return;
   }
-  const int n = seqlen - p.q_per_seq + i + 1;  // visible keys 0..pos
+  int n = seqlen - p.q_per_seq + i + 1;  // visible keys 0..pos
+  if (p.tile_stride > 1) n = ((n - 1) / 128 / p.tile_stride + 1) * 128;  // sampled row
   const uint32_t k = (uint32_t)p.k;
   if (n <= p.k) {
-    for (int j = tid; j < p.k; j += kTopkThreads) out[j] = j < n ? j : -1;
+    if (out)
+      for (int j = tid; j < p.k; j += kTopkThreads) out[j] = j < n ? j : -1;
+    if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = -INFINITY;
     return;
   }
   const float* row = p.scores + (int64_t)(blockIdx.x) * p.ld;
@@ -282,15 +297,19 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
     if (!overflow && m_run >= k) {
       const int m = (int)m_run;
       find_kth(m, k, [&](int e, int) { return cand_key[e]; }, hist, misc, tau, r_eq);
-      compact_topk(m, tau, r_eq, [&](int e, int) { return cand_key[e]; },
-                   [&](int e) { return cand_pos[e]; }, out, misc);
+      if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = key_score(tau);
+      if (out)
+        compact_topk(m, tau, r_eq, [&](int e, int) { return cand_key[e]; },
+                     [&](int e) { return cand_pos[e]; }, out, misc);
       return;
     }
     // the sample misjudged this row: exact selection over the whole row
     __syncthreads();
     find_kth(n, k, [&](int e, int) { return score_key(row[e]); }, hist, misc, tau, r_eq);
-    compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(row[e]); },
-                 [&](int e) { return e; }, out, misc);
+    if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = key_score(tau);
+    if (out)
+      compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(row[e]); },
+                   [&](int e) { return e; }, out, misc);
     return;
   }
 
@@ -322,8 +341,119 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
     __syncthreads();
   }
   find_kth(n, k, [&](int e, int) { return score_key(cache[e]); }, hist, misc, tau, r_eq);
-  compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(cache[e]); },
-               [&](int e) { return e; }, out, misc);
+  if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = key_score(tau);
+  if (out)
+    compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(cache[e]); },
+                 [&](int e) { return e; }, out, misc);
+}
+
+// ======================================================================================
+// Selection from a candidate list (the fused indexer -> top-k path)
+// ======================================================================================
+// Each window row comes with the keys the indexer's filter kept: every visible key
+// whose score reached the row's threshold, as (order-preserving key, position) in no
+// particular order. When the list holds at least k keys (and all of them: count <=
+// capacity), it contains the k largest of the row, so the exact top-k is selected
+// from it: the k-th key tau and the number r of equal keys to take (find_kth), keys
+// above tau marked in a bitmap over the row's positions, the r lowest positions of
+// the keys equal to tau marked from a second bitmap, and the marks compacted in
+// ascending order. Other rows are listed for the full (unfused) selection.
+constexpr int kCandThreads = 512;
+constexpr int kCandCap = 8192;                     // candidates per row staged in smem
+constexpr int kCandMaxWords = 4096;                // bitmap words: rows of <= 131072 keys
+
+struct CandParams {
+  const uint32_t* cand_key;  // [batch * row_count][cand_cap]
+  const int32_t* cand_pos;   // [batch * row_count][cand_cap]
+  const uint32_t* cand_cnt;  // [batch * row_count]
+  int32_t cand_cap;          // <= kCandCap
+  const int32_t* seqlens;    // [batch] or nullptr
+  int32_t max_ctx, q_per_seq, row_begin, row_count, batch, k;
+  int32_t* idx;              // [batch * q_per_seq][k]
+  int32_t* redo_rows;        // [batch * row_count] window rows left to the full path
+  uint32_t* redo_cnt;        // how many (zeroed by the caller)
+};
+
+constexpr int kCandSmemBytes =
+    kCandCap * 8 + 2 * kCandMaxWords * 4 + 2048 * 4 + 64 * 4;
+
+__global__ void __launch_bounds__(kCandThreads, 2) cand_select_kernel(CandParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(smem_raw);          // [kCandCap]
+  int32_t* cpos = reinterpret_cast<int32_t*>(ckey + kCandCap);     // [kCandCap]
+  uint32_t* sel = reinterpret_cast<uint32_t*>(cpos + kCandCap);    // [kCandMaxWords]
+  uint32_t* tie = sel + kCandMaxWords;                             // [kCandMaxWords]
+  uint32_t* hist = tie + kCandMaxWords;                            // [2048]
+  uint32_t* misc = hist + 2048;                                    // [64]
+
+  const int64_t wrow = blockIdx.x;
+  const int b = (int)(wrow / p.row_count);
+  const int i = p.row_begin + (int)(wrow - (int64_t)b * p.row_count);
+  const int64_t t = (int64_t)b * p.q_per_seq + i;
+  const int tid = threadIdx.x;
+  int32_t* out = p.idx + t * p.k;
+  const int seqlen = p.seqlens ? p.seqlens[b] : p.max_ctx;
+  if (seqlen < p.q_per_seq || seqlen > p.max_ctx) {
+    if (tid == 0) report_error(kErrBounds);
+    for (int j = tid; j < p.k; j += kCandThreads) out[j] = -1;
+    return;
+  }
+  const int n = seqlen - p.q_per_seq + i + 1;  // visible keys 0..pos
+  if (n <= p.k) {
+    for (int j = tid; j < p.k; j += kCandThreads) out[j] = j < n ? j : -1;
+    return;
+  }
+  const uint32_t m = p.cand_cnt[wrow];
+  if (m < (uint32_t)p.k || m > (uint32_t)p.cand_cap) {
+    if (tid == 0) p.redo_rows[atomicAdd(p.redo_cnt, 1u)] = (int32_t)wrow;
+    return;
+  }
+  const int words = (n + 31) >> 5;  // <= kCandMaxWords (checked on the host)
+  for (uint32_t e = tid; e < m; e += kCandThreads) {
+    ckey[e] = p.cand_key[wrow * p.cand_cap + e];
+    cpos[e] = p.cand_pos[wrow * p.cand_cap + e];
+  }
+  for (int w = tid; w < words; w += kCandThreads) sel[w] = tie[w] = 0u;
+  __syncthreads();
+  uint32_t tau, r_eq;
+  find_kth((int)m, (uint32_t)p.k, [&](int e, int) { return ckey[e]; }, hist, misc, tau, r_eq);
+  for (uint32_t e = tid; e < m; e += kCandThreads) {
+    const uint32_t key = ckey[e];
+    const int pos = cpos[e];
+    if (key > tau) atomicOr(&sel[pos >> 5], 1u << (pos & 31));
+    else if (key == tau) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+  }
+  __syncthreads();
+  // the r_eq lowest positions among the keys equal to tau: an ordered scan of the
+  // tie bitmap (each thread owns consecutive words)
+  const int per = (words + kCandThreads - 1) / kCandThreads;
+  const int w0 = tid * per;
+  uint32_t cnt = 0;
+  for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(tie[w]);
+  uint32_t before = block_exclusive_scan(cnt, misc, misc + 32);
+  for (int w = w0; w < w0 + per && w < words; ++w) {
+    uint32_t bits = tie[w];
+    while (bits) {
+      const uint32_t bit = bits & (~bits + 1u);
+      if (before < r_eq) sel[w] |= bit;
+      ++before;
+      bits ^= bit;
+    }
+  }
+  __syncthreads();
+  // ascending compaction of the selection (exactly k marks)
+  cnt = 0;
+  for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(sel[w]);
+  uint32_t o = block_exclusive_scan(cnt, misc, misc + 32);
+  for (int w = w0; w < w0 + per && w < words; ++w) {
+    uint32_t bits = sel[w];
+    while (bits) {
+      const int bpos = __ffs(bits) - 1;
+      if (o < (uint32_t)p.k) out[o] = w * 32 + bpos;
+      ++o;
+      bits &= bits - 1u;
+    }
+  }
 }
 
 }  // namespace dsa

@@ -83,6 +83,14 @@ SIGNATURES = {
     "dsa_mha_prefill": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(KvDescC),
                                        ctypes.POINTER(QDescC), ctypes.c_int32, ctypes.c_float, _P,
                                        ctypes.c_size_t, _P, _P, _P, _P]),
+    "dsa_fused_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
+                                                   ctypes.c_int32]),
+    "dsa_select_fused": (ctypes.c_int, [_P, _P, _P, _P, ctypes.POINTER(KvDescC),
+                                        ctypes.POINTER(QDescC), ctypes.c_int32, ctypes.c_int32, _P,
+                                        ctypes.c_size_t, _P, _P]),
+    "dsa_forward_fused": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.POINTER(KvDescC),
+                                         ctypes.POINTER(QDescC), ctypes.c_int32, ctypes.c_float,
+                                         ctypes.c_int32, _P, ctypes.c_size_t, _P, _P, _P, _P]),
     "dsa_get_device_error": (ctypes.c_int, [_P]),
     "dsa_set_wait_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "dsa_selftest_wait_timeout": (ctypes.c_int, [_P]),
@@ -274,6 +282,51 @@ def dsa_forward_noalloc(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_p
                                      _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k,
                                      float(scale), _ptr(idx_out), _ptr(out), _ptr(lse),
                                      _stream(stream)), "dsa_forward_noalloc")
+    return out, lse, idx_out
+
+
+# ---- fused indexer -> top-k (no stored score rows) -------------------------------------
+
+
+def dsa_fused_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None) -> int:
+    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows)
+    return int(lib().dsa_fused_workspace_size(ctypes.byref(kvd), ctypes.byref(qd), k))
+
+
+def dsa_select_fused(q_idx, w, k_idx, k_scale, kv: KvLayout, q_per_seq: int, k: int,
+                     cand_cap: int = 0, idx=None, workspace=None, rows=None, stream=None):
+    """Selected positions [T, k] without stored score rows (include/dsa.h)."""
+    T = q_idx.shape[0]
+    if idx is None:
+        idx = torch.empty(T, k, dtype=torch.int32, device=q_idx.device)
+    if workspace is None:
+        nbytes = dsa_fused_workspace_size(kv, T, q_per_seq, k, rows)
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q_idx.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    _check(lib().dsa_select_fused(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale),
+                                  ctypes.byref(kvd), ctypes.byref(qd), k, int(cand_cap),
+                                  _ptr(workspace), workspace.numel(), _ptr(idx), _stream(stream)),
+           "dsa_select_fused")
+    return idx
+
+
+def dsa_forward_fused(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_per_seq: int,
+                      k: int, scale: float, cand_cap: int = 0, workspace=None, idx_out=None,
+                      out=None, lse=None, rows=None, stream=None):
+    T = q.shape[0]
+    if workspace is None:
+        nbytes = dsa_fused_workspace_size(kv, T, q_per_seq, k, rows)
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    _check(lib().dsa_forward_fused(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q),
+                                   _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k,
+                                   float(scale), int(cand_cap), _ptr(workspace),
+                                   workspace.numel(), _ptr(idx_out), _ptr(out), _ptr(lse),
+                                   _stream(stream)), "dsa_forward_fused")
     return out, lse, idx_out
 
 
