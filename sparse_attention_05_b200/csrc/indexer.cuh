@@ -47,7 +47,8 @@ constexpr int kIdxStageBytes = kIdxTile * kIdxDim;  // 16 KB of e4m3
 constexpr int kIdxQBufBytes = 4 * kIdxHeads * kIdxDim;  // G <= 4 rows x 64 heads x 128 B
 constexpr int kIdxSmemBytes =
     1024 /*align slack*/ + kIdxStages * kIdxStageBytes + 2 * kIdxQBufBytes +
-    2 * 4 * kIdxHeads * 4 /*wq*/ + 512 /*barriers etc*/ + 512 /*share + scan scratch*/;
+    2 * 4 * kIdxHeads * 4 /*wq*/ + 512 /*barriers etc*/ + 512 /*share + scan scratch*/ +
+    2 * 4 * 256 * 4 /*filter mode: candidate keys staged for one tile*/;
 constexpr int kIdxMaxAcc = 8;  // TMEM accumulators: 512 / N, at most 8
 
 struct IndexerParams {
@@ -217,6 +218,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   IdxShare* share = reinterpret_cast<IdxShare*>(tmem_holder + 4);
   uint32_t* scan_scratch = reinterpret_cast<uint32_t*>(share + 1) + 4;  // 8-B aligned, 32 x i64
+  // filter mode: [2 tiles][4 rows][256 epilogue threads] keys awaiting their slots
+  uint32_t* cstage = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + 1024);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = kIdxHeads * p.G;
@@ -426,6 +429,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const int wg = (warp - 4) >> 2;    // warpgroup: owns TMEM accumulator `wg`
     const int quad = warp & 3;         // TMEM lane quadrant of this warp
     const int e = quad * 32 + lane;    // key within the tile == TMEM lane
+    const int et = tid - 4 * 32;       // 0..255 among the epilogue threads
+    int cpar = 0;                      // filter mode: staging buffer of the next tile
     uint32_t it = 0, un = 0;
     if (blockIdx.x == 0 && wg == 0) {  // sequences whose length cannot hold their rows
       for (int b = e; b < p.batch; b += 128) {
@@ -460,6 +465,28 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       };
       int pf_kt = -1;  // the tile whose scale is already in flight (this warpgroup's next)
       float pf_ks = 0.f;
+      // Filter mode: a tile's candidates reserve their slots (one atomic per warp and
+      // row) after its rows are reduced, and are written one tile later, so the
+      // atomic's round trip overlaps the next tile instead of stalling the warp.
+      const int64_t orow0 = (int64_t)U.b * p.row_count + (U.i0 - p.row_begin);
+      uint32_t pend_bal[4] = {0u, 0u, 0u, 0u}, pend_base[4] = {0u, 0u, 0u, 0u};
+      uint32_t pend_bits = 0;
+      int pend_s = 0, pend_par = 0;
+      auto flush = [&]() {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t bal = pend_bal[g];
+          if (bal) {  // warp-uniform
+            const uint32_t base = __shfl_sync(0xffffffffu, pend_base[g], __ffs(bal) - 1);
+            const uint32_t slot = base + __popc(bal & ((1u << lane) - 1u));
+            if (((pend_bits >> g) & 1u) && slot < (uint32_t)p.cand_cap) {
+              p.cand_key[(orow0 + g) * p.cand_cap + slot] = cstage[((pend_par * 4 + g) << 8) + et];
+              p.cand_pos[(orow0 + g) * p.cand_cap + slot] = pend_s;
+            }
+          }
+          pend_bal[g] = 0u;
+        }
+      };
       bool ok = true;
       for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
         if ((int)(it & 1) != wg) continue;  // the other warpgroup's tile
@@ -481,6 +508,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         // hides behind the ReLU / weighted head sum.
         const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * N;
         uint32_t ca[32], cb[32];
+        uint32_t take_bits = 0;  // filter mode: rows that keep this thread's key
         tmem_ld32u(tcol, ca);
         tmem_wait_ld_fence(ca);
         for (int gi = 0; gi < U.nrows; ++gi) {
@@ -507,25 +535,33 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           const int64_t orow = (int64_t)U.b * p.row_count + (U.i0 - p.row_begin) + gi;
           if (!p.thr) {
             p.scores[orow * p.ld + kt * kIdxTile + e] = out;
-          } else {  // filter mode: append (key, position) when the score reaches thr
+          } else {  // filter mode: note the key; its slot is reserved after the rows
             const bool take = s <= pos0 + gi && out >= thr_row[gi];
-            const uint32_t ballot = __ballot_sync(0xffffffffu, take);
-            if (ballot) {
-              uint32_t base = 0;
-              if (lane == __ffs(ballot) - 1) base = atomicAdd(p.cand_cnt + orow, __popc(ballot));
-              base = __shfl_sync(0xffffffffu, base, __ffs(ballot) - 1);
-              const uint32_t slot = base + __popc(ballot & ((1u << lane) - 1u));
-              if (take && slot < (uint32_t)p.cand_cap) {
-                p.cand_key[orow * p.cand_cap + slot] = score_key(out);
-                p.cand_pos[orow * p.cand_cap + slot] = s;
-              }
-            }
+            take_bits |= (take ? 1u : 0u) << gi;
+            cstage[((cpar * 4 + gi) << 8) + et] = score_key(out);
           }
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&tempty[ab]));
+        if (p.thr) {
+          flush();  // the previous tile's candidates: their slots have arrived by now
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t bal =
+                __ballot_sync(0xffffffffu, g < U.nrows && ((take_bits >> g) & 1u));
+            pend_bal[g] = bal;
+            pend_base[g] = 0u;
+            if (bal && lane == __ffs(bal) - 1)
+              pend_base[g] = atomicAdd(p.cand_cnt + orow0 + g, __popc(bal));
+          }
+          pend_bits = take_bits;
+          pend_s = s;
+          pend_par = cpar;
+          cpar ^= 1;
+        }
       }
       if (!ok) break;
+      if (p.thr) flush();  // the unit's last tile
       mbar_arrive(smem_u32(&qempty[qb]));
       ++un;
     }
