@@ -244,6 +244,25 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------------------
+def mla_split_launches(rows: int, k: int, scratch_bytes: int) -> int:
+    """Kernel launches of one dsa_sparse_mla_fwd_ws call: the attention, plus the
+    segment merge when the library's rule splits the rows of a last wave that is at
+    most half full (clusters of 2 SMs; 2..8 segments of >= 6 blocks of 48 keys, as
+    many as the scratch holds at 256.5 KB each). Used for the launch count only."""
+    wave = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    tail = rows % wave if wave >= 2 and rows > 0 else 0
+    if tail == 0:
+        return 1
+    nb = -(-k // 48)
+    s = min(wave // tail, 8, nb // 6)
+    while s >= 2 and tail * s * (128 * 512 * 4 + 128 * 4) > scratch_bytes:
+        s -= 1
+    if s < 2:
+        return 1
+    bps = -(-nb // s)
+    return 2 if -(-nb // bps) >= 2 else 1
+
+
 class Runner:
     """Holds the device buffers of one workload and runs one step of the path
     through the library's stage calls (the same launches dsa_forward makes)."""
@@ -262,17 +281,26 @@ class Runner:
         elif rows >= 4:
             rows &= ~3
         self.chunks = [(r0, min(rows, p.q_per_seq - r0)) for r0 in range(0, p.q_per_seq, rows)]
-        self.scores = torch.empty(B * rows, self.ld, dtype=torch.float32, device=p.q.device)
+        # the score rows, whose space the sparse MLA then uses as its split scratch
+        # (as in dsa_forward's workspace)
+        nscore = B * rows * self.ld * 4
+        self.ws = torch.empty(max(nscore, dsa.dsa_sparse_mla_workspace_size()), dtype=torch.uint8,
+                              device=p.q.device)
+        self.scores = self.ws[:nscore].view(torch.float32).view(B * rows, self.ld)
         self.idx = torch.empty(T, k, dtype=torch.int32, device=p.q.device)
         self.out = torch.empty(T, 128, 512, dtype=torch.bfloat16, device=p.q.device)
         self.lse = torch.empty(T, 128, dtype=torch.float32, device=p.q.device)
-        self.launches_per_step = 2 * len(self.chunks) + 1
+        self.mla_ws = self.ws
         self.with_kl = with_kl
         if with_kl:
             if len(self.chunks) > 1:
                 raise SystemExit("--kl needs every score row in one chunk (not this workload)")
             self.kl = torch.empty(T, dtype=torch.float32, device=p.q.device)
-            self.launches_per_step += 1
+            # the KL term reads the score rows after the attention: keep them intact
+            self.mla_ws = torch.empty(dsa.dsa_sparse_mla_workspace_size(), dtype=torch.uint8,
+                                      device=p.q.device)
+        self.launches_per_step = (2 * len(self.chunks) + mla_split_launches(T, k, self.mla_ws.numel())
+                                  + (1 if with_kl else 0))
 
     def step(self, ev=None):
         d, p = self.dsa, self.p
@@ -290,8 +318,8 @@ class Runner:
                 ev["topk"].append(_record())
         if ev is not None:
             ev["sparse_mla"].append(_record())
-        d.dsa_sparse_mla_fwd(p.q, p.kv, self.kv, p.q_per_seq, self.idx, p.scale, out=self.out,
-                             lse=self.lse)
+        d.dsa_sparse_mla_fwd_ws(p.q, p.kv, self.kv, p.q_per_seq, self.idx, p.scale,
+                                workspace=self.mla_ws, out=self.out, lse=self.lse)
         if ev is not None:
             ev["sparse_mla"].append(_record())
         if self.with_kl:  # the indexer's KL loss term over the selected sets
@@ -382,9 +410,11 @@ class FusedRunner(Runner):
         nbytes = d.dsa_fused_workspace_size(self.kv, p.num_q, p.q_per_seq, k)
         self.ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=p.q.device)
         self.scores = None  # never materialised
+        self.mla_ws = self.ws  # dead once the selection is done (as in dsa_forward_fused)
         # per chunk: sampled indexer, threshold top-k, filtering indexer, selection
         per = max(1, (2 << 30) // (p.batch * (self.ld // 8 * 4 + 12 + 8192 * 8)))
-        self.launches_per_step = 4 * (-(-p.q_per_seq // per)) + 1
+        self.launches_per_step = (4 * (-(-p.q_per_seq // per))
+                                  + mla_split_launches(p.num_q, k, self.ws.numel()))
 
     def step(self, ev=None):
         d, p = self.dsa, self.p
@@ -395,8 +425,8 @@ class FusedRunner(Runner):
         if ev is not None:
             ev["select_fused"].append(_record())
             ev["sparse_mla"].append(_record())
-        d.dsa_sparse_mla_fwd(p.q, p.kv, self.kv, p.q_per_seq, self.idx, p.scale, out=self.out,
-                             lse=self.lse)
+        d.dsa_sparse_mla_fwd_ws(p.q, p.kv, self.kv, p.q_per_seq, self.idx, p.scale,
+                                workspace=self.mla_ws, out=self.out, lse=self.lse)
         if ev is not None:
             ev["sparse_mla"].append(_record())
 

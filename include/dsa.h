@@ -135,6 +135,28 @@ DSA_API dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv_cache, con
                                 const dsa_q_desc_t* qd, const int32_t* idx, int32_t k,
                                 float scale, void* out, float* lse, dsa_stream_t stream);
 
+/* dsa_sparse_mla_fwd with a scratch buffer that lets the call balance its last wave.
+ * The rows run as one 2-CTA cluster each, (SMs / 2) clusters at a time; when the
+ * last wave would hold at most half as many rows as a full one, each of its rows is
+ * split into 2..8 key segments (consecutive parts of its idx row, at least 288
+ * entries each) run as clusters of their own, and a second kernel merges the
+ * segments: LSE = ln sum_s e^{LSE_s}, o = sum_s e^{LSE_s - LSE} o_s. Results agree
+ * with dsa_sparse_mla_fwd up to fp32 rounding (not bit for bit).
+ *  workspace  device, 256-byte aligned, workspace_bytes long, or NULL / 0 (then no
+ *             row is split and the call is dsa_sparse_mla_fwd). The library writes
+ *             it during the call (stream order) and keeps nothing in it afterwards.
+ *             Fewer bytes than dsa_sparse_mla_workspace_size() only allow fewer
+ *             segments. Other arguments as dsa_sparse_mla_fwd. */
+DSA_API dsa_status_t dsa_sparse_mla_fwd_ws(const void* q, const void* kv_cache,
+                                           const dsa_kv_desc_t* kv, const dsa_q_desc_t* qd,
+                                           const int32_t* idx, int32_t k, float scale,
+                                           void* workspace, size_t workspace_bytes, void* out,
+                                           float* lse, dsa_stream_t stream);
+
+/* Bytes of scratch with which dsa_sparse_mla_fwd_ws may split every row it would
+ * split on this device (at most (SMs / 2) segments of 256.5 KB). */
+DSA_API size_t dsa_sparse_mla_workspace_size(void);
+
 /* Indexer training target and KL loss term (report §2.1: the main attention summed
  * over all heads and L1-normalised along the sequence is the target p_{t,:}; the
  * indexer is trained with KL(p_{t,:} || Softmax(I_{t,:})), over every visible key in
@@ -165,8 +187,10 @@ DSA_API size_t dsa_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q
  * dsa_workspace_size() bytes let the score rows go in chunks of up to 2 GiB. A
  * smaller workspace is accepted down to the indices plus one score row per
  * sequence; the rows are then processed in smaller chunks. Too small a
- * workspace returns DSA_ERR_WORKSPACE. idx_out (int32 [T][k]) receives the
- * selection when not NULL. */
+ * workspace returns DSA_ERR_WORKSPACE. Once the selection is done, the space of the
+ * score rows serves the sparse MLA as dsa_sparse_mla_fwd_ws's scratch (split rows of
+ * a partly filled last wave); dsa_workspace_size() includes what that needs.
+ * idx_out (int32 [T][k]) receives the selection when not NULL. */
 DSA_API dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
                          const float* k_scale, const void* q, const void* kv_cache,
                          const dsa_kv_desc_t* kv, const dsa_q_desc_t* qd, int32_t k,
@@ -229,9 +253,11 @@ DSA_API dsa_status_t dsa_select_fused(const void* q_idx, const float* w, const v
                                       void* workspace, size_t workspace_bytes, int32_t* idx,
                                       dsa_stream_t stream);
 
-/* dsa_forward with the fused selection: dsa_select_fused then dsa_sparse_mla_fwd.
+/* dsa_forward with the fused selection: dsa_select_fused then dsa_sparse_mla_fwd_ws.
  * Arguments as dsa_forward plus cand_cap; the workspace holds the indices (unless
- * idx_out is given) followed by dsa_select_fused's workspace. */
+ * idx_out is given) followed by dsa_select_fused's workspace, which then serves as
+ * the sparse MLA's split scratch (dsa_fused_workspace_size() includes what that
+ * needs). */
 DSA_API dsa_status_t dsa_forward_fused(const void* q_idx, const float* w, const void* k_idx,
                                        const float* k_scale, const void* q,
                                        const void* kv_cache, const dsa_kv_desc_t* kv,

@@ -155,8 +155,11 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(indexer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kIdxSmemBytes);
+    attr_err = cudaFuncSetAttribute(indexer_kernel<false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmemBytes);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(indexer_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   CUtensorMap tm;
@@ -193,14 +196,52 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   // every CTA takes an equal share of all key tiles (at most one CTA per tile)
   const int64_t max_tiles = (int64_t)p.num_groups * ((g.max_ctx + kIdxTile - 1) / kIdxTile);
   const int grid = (int)std::min<int64_t>(max_tiles, num_sms());
-  indexer_kernel<<<grid, kIdxThreads, kIdxSmemBytes, stream>>>(p, tm);
+  if (p.thr) {
+    indexer_kernel<true><<<grid, kIdxThreads, kIdxSmemBytes, stream>>>(p, tm);
+  } else {
+    indexer_kernel<false><<<grid, kIdxThreads, kIdxSmemBytes, stream>>>(p, tm);
+  }
   return cuda_status(cudaGetLastError());
 }
 
 // ---- sparse MLA launch --------------------------------------------------------------
+// How the rows of one call are spread over clusters. A call's clusters run in waves
+// of (SMs / 2) clusters; when the last wave is at most half full, its rows are split
+// into as many key segments as fill it (at least 6 key blocks each, at most
+// kMlaMaxSeg, and only as many as the scratch holds), and merged afterwards.
+struct MlaSplit {
+  int64_t n_whole = 0, n_split = 0;
+  int nseg = 1, seg_keys = 0;
+};
+constexpr size_t kMlaPartBytes = (size_t)kMlaHeads * kMlaDv * 4 + kMlaHeads * 4;
+
+MlaSplit plan_mla_split(int64_t rows, int k, size_t scratch_bytes) {
+  MlaSplit sp;
+  sp.n_whole = rows;
+  sp.seg_keys = k;
+  const int64_t wave = num_sms() / 2;
+  if (wave < 2 || rows <= 0) return sp;
+  const int64_t tail = rows % wave;
+  const int nb = (k + kMlaBlk - 1) / kMlaBlk;
+  if (tail == 0) return sp;
+  int s = (int)std::min<int64_t>(wave / tail, kMlaMaxSeg);
+  s = std::min(s, nb / 6);
+  while (s >= 2 && (size_t)tail * s * kMlaPartBytes > scratch_bytes) --s;
+  if (s < 2) return sp;
+  const int bps = (nb + s - 1) / s;  // blocks per segment; every segment non-empty
+  sp.nseg = (nb + bps - 1) / bps;
+  if (sp.nseg < 2) return sp;
+  sp.seg_keys = bps * kMlaBlk;
+  sp.n_whole = rows - tail;
+  sp.n_split = tail;
+  return sp;
+}
+
+// `scratch` (256-B aligned, may be null) holds the segments' partial outputs.
 dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geometry& g,
                                const int32_t* idx, int k, float scale, void* out, float* lse,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, void* scratch = nullptr,
+                               size_t scratch_bytes = 0) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -234,8 +275,19 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
   p.row_count = g.row_count;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns.load();
+  const int64_t rows = (int64_t)g.batch * g.row_count;
+  if (rows == 0) return DSA_OK;
+  const MlaSplit sp = plan_mla_split(rows, k, scratch ? scratch_bytes : 0);
+  p.n_whole = sp.n_whole;
+  p.nseg = sp.nseg;
+  p.seg_keys = sp.seg_keys;
+  const int64_t slots = sp.n_split * sp.nseg;
+  if (slots > 0) {
+    p.part_o = reinterpret_cast<float*>(scratch);
+    p.part_lse = p.part_o + slots * kMlaHeads * kMlaDv;
+  }
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(2 * (int64_t)g.batch * g.row_count), 1, 1);
+  cfg.gridDim = dim3((unsigned)(2 * (sp.n_whole + slots)), 1, 1);
   cfg.blockDim = dim3(kMlaThreads, 1, 1);
   cfg.dynamicSmemBytes = kMlaSmemBytes;
   cfg.stream = stream;
@@ -246,7 +298,20 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, sparse_mla_kernel, p, tm));
+  st = cuda_status(cudaLaunchKernelEx(&cfg, sparse_mla_kernel, p, tm));
+  if (st != DSA_OK || slots == 0) return st;
+  MlaCombineParams c{};
+  c.part_o = p.part_o;
+  c.part_lse = p.part_lse;
+  c.out = p.out;
+  c.lse = lse;
+  c.n_whole = sp.n_whole;
+  c.nseg = sp.nseg;
+  c.row_begin = g.row_begin;
+  c.row_count = g.row_count;
+  c.q_per_seq = g.q_per_seq;
+  mla_combine_kernel<<<dim3((unsigned)sp.n_split, kMlaHeads / 8), 256, 0, stream>>>(c);
+  return cuda_status(cudaGetLastError());
 }
 
 // ---- indexer KL launch -------------------------------------------------------------
@@ -633,11 +698,32 @@ dsa_status_t dsa_sparse_mla_fwd(const void* q, const void* kv_cache, const dsa_k
   return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, (cudaStream_t)stream);
 }
 
+dsa_status_t dsa_sparse_mla_fwd_ws(const void* q, const void* kv_cache, const dsa_kv_desc_t* kv,
+                                   const dsa_q_desc_t* qd, const int32_t* idx, int32_t k,
+                                   float scale, void* workspace, size_t workspace_bytes,
+                                   void* out, float* lse, dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, qd, &g);
+  if (st != DSA_OK) return st;
+  if (!q || !kv_cache || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!(scale > 0.f) || !(scale < 1e30f)) return DSA_ERR_INVALID_ARG;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+  return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, (cudaStream_t)stream,
+                           workspace, workspace ? workspace_bytes : 0);
+}
+
+size_t dsa_sparse_mla_workspace_size(void) { return (size_t)(num_sms() / 2) * kMlaPartBytes; }
+
 size_t dsa_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k) {
   Geometry g;
   if (check_geometry(kv, q, &g) != DSA_OK || k < 1 || k > kMaxK) return 0;
   const ForwardPlan f = plan_forward(g, k, true);
-  return f.idx_bytes + f.score_bytes;
+  // after the selection the score space holds the sparse MLA's split rows
+  const MlaSplit sp = plan_mla_split((int64_t)g.batch * g.row_count, k, SIZE_MAX);
+  const size_t part_bytes = (size_t)(sp.n_split * sp.nseg) * kMlaPartBytes;
+  return f.idx_bytes + std::max(f.score_bytes, align256(part_bytes));
 }
 
 dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
@@ -680,7 +766,10 @@ dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
     st = launch_topk(scores, f.ld, g, r0, rc, k, idx, s);
     if (st != DSA_OK) return st;
   }
-  return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, s);
+  // the score rows are dead once the last top-k has run (stream order): their
+  // space holds the partial outputs of split rows
+  return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, s, scores,
+                           workspace_bytes - f.idx_bytes);
 }
 
 dsa_status_t dsa_forward_noalloc(const void* q_idx, const float* w, const void* k_idx,
@@ -861,8 +950,10 @@ size_t dsa_fused_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, 
   Geometry g;
   if (check_geometry(kv, q, &g) != DSA_OK || k < 1 || k > kMaxK) return 0;
   const FusedPlan f = plan_fused(g, k, true, 0);
-  return f.idx_bytes + f.fallback_bytes +
-         (size_t)f.chunk_rows * g.batch * f.row_bytes + 8 * 256;
+  const size_t sel = f.fallback_bytes + (size_t)f.chunk_rows * g.batch * f.row_bytes + 8 * 256;
+  // dsa_forward_fused: after the selection the same space holds the split rows
+  const MlaSplit sp = plan_mla_split((int64_t)g.batch * g.row_count, k, SIZE_MAX);
+  return f.idx_bytes + std::max(sel, align256((size_t)(sp.n_split * sp.nseg) * kMlaPartBytes));
 }
 
 dsa_status_t dsa_select_fused(const void* q_idx, const float* w, const void* k_idx,
@@ -921,7 +1012,10 @@ dsa_status_t dsa_forward_fused(const void* q_idx, const float* w, const void* k_
                         reinterpret_cast<uint8_t*>(workspace) + idx_bytes,
                         workspace_bytes - idx_bytes, idx, stream);
   if (st != DSA_OK) return st;
-  return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, (cudaStream_t)stream);
+  // the selection's workspace is dead now: it holds the split rows' partial outputs
+  return launch_sparse_mla(q, kv_cache, g, idx, k, scale, out, lse, (cudaStream_t)stream,
+                           reinterpret_cast<uint8_t*>(workspace) + idx_bytes,
+                           workspace_bytes - idx_bytes);
 }
 
 dsa_status_t dsa_selftest_wait_timeout(dsa_stream_t stream) {

@@ -197,6 +197,9 @@ __device__ void idx_share(const IndexerParams& p, IdxShare* out, uint32_t* scrat
   __syncthreads();
 }
 
+// kFilter: the fused selection's filter mode (thr, cand_* set; no score rows); the
+// plain instantiation carries none of its code.
+template <bool kFilter>
 __global__ void __launch_bounds__(kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ IndexerParams p,
                    const __grid_constant__ CUtensorMap tm_keys) {
@@ -447,7 +450,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       const int pos0 = U.seqlen - p.q_per_seq + U.i0;  // position of the group's first row
       const int pos_max = pos0 + U.nrows - 1;
       float thr_row[4] = {0.f, 0.f, 0.f, 0.f};  // filter mode: the rows' thresholds
-      if (p.thr)
+      if (kFilter)
         for (int gi = 0; gi < U.nrows; ++gi)
           thr_row[gi] = __ldg(p.thr + (int64_t)U.b * p.row_count + (U.i0 - p.row_begin) + gi);
       // this thread's key scale of tile kt (0 past the last visible key or behind
@@ -533,7 +536,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           const float acc = (a0 + a1) + (a2 + a3);
           const float out = (s <= pos0 + gi) ? ks * acc : -INFINITY;
           const int64_t orow = (int64_t)U.b * p.row_count + (U.i0 - p.row_begin) + gi;
-          if (!p.thr) {
+          if (!kFilter) {
             p.scores[orow * p.ld + kt * kIdxTile + e] = out;
           } else {  // filter mode: note the key; its slot is reserved after the rows
             const bool take = s <= pos0 + gi && out >= thr_row[gi];
@@ -543,7 +546,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&tempty[ab]));
-        if (p.thr) {
+        if (kFilter) {
           flush();  // the previous tile's candidates: their slots have arrived by now
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
@@ -561,7 +564,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
       }
       if (!ok) break;
-      if (p.thr) flush();  // the unit's last tile
+      if (kFilter) flush();  // the unit's last tile
       mbar_arrive(smem_u32(&qempty[qb]));
       ++un;
     }

@@ -55,6 +55,12 @@
 //                          with a lazy rescale of O (only when the running max
 //                          grows by more than 8), which the owner's factor
 //                          carries to the peer's half of O.
+//
+// Clusters run in waves of (SMs / 2). When a call's last wave would be at most half
+// full, the host may split each of its rows into key segments (consecutive parts of
+// the row's selection, whole 48-key blocks) run as clusters of their own; each
+// writes its segment's normalised output in fp32 and its LSE, and
+// mla_combine_kernel merges them (softmax over a union of disjoint sets).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -124,6 +130,16 @@ struct MlaParams {
   int64_t cache_rows;
   float scale_log2;            // scale * log2(e)
   uint64_t timeout_ns;
+  // Rows of a last, partly filled wave may be split into key segments: clusters
+  // [0, n_whole) take whole rows (cluster c = window row c); cluster n_whole + j
+  // takes segment j % nseg (keys [seg_keys (j % nseg), + seg_keys) of the row's
+  // selection) of window row n_whole + j / nseg and writes that segment's
+  // normalised output (fp32) and LSE to slot j of part_o / part_lse, which
+  // mla_combine_kernel merges.
+  int64_t n_whole;
+  int32_t nseg, seg_keys;
+  float* part_o;               // [slots][128][512]
+  float* part_lse;             // [slots][128]
 };
 
 __global__ void __launch_bounds__(kMlaThreads, 1)
@@ -159,13 +175,22 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
-  const int64_t local = blockIdx.x >> 1;  // query row within the window
+  const int64_t cl = blockIdx.x >> 1;  // cluster
+  int64_t local = cl;                  // query row within the window
+  int64_t part = -1;                   // partial-output slot of a row segment
+  int e0 = 0, e1 = p.k;                // this cluster's entries of the row's selection
+  if (cl >= p.n_whole) {
+    part = cl - p.n_whole;
+    local = p.n_whole + part / p.nseg;
+    e0 = (int)(part % p.nseg) * p.seg_keys;
+    e1 = min(p.k, e0 + p.seg_keys);
+  }
   const int b = (int)(local / p.row_count);
   const int qi = p.row_begin + (int)(local - (int64_t)b * p.row_count);
   const int64_t t = (int64_t)b * p.q_per_seq + qi;  // global query row
   const int d0 = 256 * (int)rank;        // first value dim (and first key dim) of this CTA
   const int r0 = 512 + 32 * (int)rank;   // this CTA's quarter of the rope dims
-  const int nblk = (p.k + kMlaBlk - 1) / kMlaBlk;
+  const int nblk = (e1 - e0 + kMlaBlk - 1) / kMlaBlk;
 
   if (tid == 0) {
     for (int i = 0; i < kMlaStages; ++i) {
@@ -232,7 +257,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 #pragma unroll
       for (int i = 0; i < 6; ++i) {
         const int e = c * kMlaResolve + 32 * i + lane;
-        sel[i] = e < p.k ? __ldg(p.idx + t * p.k + e) : -1;
+        sel[i] = e0 + e < e1 ? __ldg(p.idx + t * p.k + e0 + e) : -1;
         if (!(seq_ok && sel[i] >= 0 && sel[i] <= pos)) sel[i] = -1;
       }
       if (p.paged) {
@@ -629,15 +654,35 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         // the peer normalises its half of these heads' rows with the same sum
         st_async_u32(mapa_shared(smem_u32(sLfin), peer) + hl * 4, __float_as_uint(lt),
                      mapa_shared(smem_u32(lfull), peer));
-        if (all_ok)
-          p.lse[t * kMlaHeads + h] = lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994531f
-                                              : -INFINITY;
+        if (all_ok) {
+          const float lse_h =
+              lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
+          if (part < 0) {
+            p.lse[t * kMlaHeads + h] = lse_h;
+          } else {
+            p.part_lse[part * kMlaHeads + h] = lse_h;
+          }
+        }
       }
     } else {
       lt_ok = warp_wait<true>(smem_u32(lfull), 0, TO, abort_flag) && all_ok;
       if (lt_ok) lt = reinterpret_cast<const float*>(sLfin)[hl];
     }
-    if (lt_ok && nblk > 0) {
+    if (lt_ok && nblk > 0 && part >= 0) {  // a row segment: fp32 for the merge
+      const float inv = lt > 0.f ? 1.0f / lt : 0.f;
+      float* prow = p.part_o + (part * kMlaHeads + h) * kMlaDv + d0 + hf * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(tO + hf * 128 + c * 32 + lane_off, o);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(prow + c * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv,
+                               o[4 * q + 3] * inv);
+      }
+    } else if (lt_ok && nblk > 0) {
       const float inv = lt > 0.f ? 1.0f / lt : 0.f;
       __nv_bfloat16* orow = p.out + (t * kMlaHeads + h) * kMlaDv + d0 + hf * 128;
 #pragma unroll 1
@@ -667,6 +712,69 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, kMlaTmemCols);
   }
+}
+
+// Merge of a row's key segments (the same attention, split over disjoint parts of
+// S_t): with segment LSEs l_s and normalised outputs o_s,
+//   LSE = ln sum_s e^{l_s},   o = sum_s e^{l_s - LSE} o_s,
+// and LSE = -inf, o = 0 when no segment holds a valid key (as for a whole row).
+constexpr int kMlaMaxSeg = 8;
+struct MlaCombineParams {
+  const float* part_o;  // [slots][128][512]
+  const float* part_lse;  // [slots][128]
+  __nv_bfloat16* out;
+  float* lse;
+  int64_t n_whole;
+  int32_t nseg, row_begin, row_count, q_per_seq;
+};
+
+// grid (split rows, 16), 256 threads: warp = one of 8 heads, lane = 16 value dims
+__global__ void __launch_bounds__(256) mla_combine_kernel(const __grid_constant__ MlaCombineParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t j = blockIdx.x;
+  const int h = blockIdx.y * 8 + warp;
+  const int64_t local = p.n_whole + j;
+  const int b = (int)(local / p.row_count);
+  const int qi = p.row_begin + (int)(local - (int64_t)b * p.row_count);
+  const int64_t t = (int64_t)b * p.q_per_seq + qi;
+  float l[kMlaMaxSeg];
+  float m = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < kMlaMaxSeg; ++s) {
+    l[s] = s < p.nseg ? __ldg(p.part_lse + (j * p.nseg + s) * kMlaHeads + h) : -INFINITY;
+    m = fmaxf(m, l[s]);
+  }
+  float o[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) o[i] = 0.f;
+  float lse_t = -INFINITY;
+  if (m != -INFINITY) {
+    float sum = 0.f;
+#pragma unroll
+    for (int s = 0; s < kMlaMaxSeg; ++s) sum += s < p.nseg ? expf(l[s] - m) : 0.f;
+    lse_t = m + logf(sum);
+#pragma unroll
+    for (int s = 0; s < kMlaMaxSeg; ++s) {
+      const float a = s < p.nseg ? expf(l[s] - lse_t) : 0.f;
+      if (a == 0.f) continue;  // warp-uniform: past nseg, or an empty or negligible segment
+      const float4* src = reinterpret_cast<const float4*>(
+          p.part_o + ((j * p.nseg + s) * kMlaHeads + h) * kMlaDv + lane * 16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 v = __ldg(src + q);
+        o[4 * q] = fmaf(a, v.x, o[4 * q]);
+        o[4 * q + 1] = fmaf(a, v.y, o[4 * q + 1]);
+        o[4 * q + 2] = fmaf(a, v.z, o[4 * q + 2]);
+        o[4 * q + 3] = fmaf(a, v.w, o[4 * q + 3]);
+      }
+    }
+  }
+  uint4* dst = reinterpret_cast<uint4*>(p.out + (t * kMlaHeads + h) * kMlaDv + lane * 16);
+  dst[0] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                      pack_bf16x2(o[6], o[7]));
+  dst[1] = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]),
+                      pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
+  if (lane == 0) p.lse[t * kMlaHeads + h] = lse_t;
 }
 
 }  // namespace dsa

@@ -60,6 +60,10 @@ SIGNATURES = {
                                 ctypes.POINTER(QDescC), ctypes.c_int32, _P, _P]),
     "dsa_sparse_mla_fwd": (ctypes.c_int, [_P, _P, ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
                                           _P, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
+    "dsa_sparse_mla_fwd_ws": (ctypes.c_int, [_P, _P, ctypes.POINTER(KvDescC),
+                                             ctypes.POINTER(QDescC), _P, ctypes.c_int32,
+                                             ctypes.c_float, _P, ctypes.c_size_t, _P, _P, _P]),
+    "dsa_sparse_mla_workspace_size": (ctypes.c_size_t, []),
     "dsa_indexer_kl": (ctypes.c_int, [_P, _P, ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
                                       _P, ctypes.c_int32, ctypes.c_float, _P, _P, ctypes.c_int64,
                                       _P, _P]),
@@ -223,6 +227,34 @@ def dsa_sparse_mla_fwd(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale: fl
     _check(lib().dsa_sparse_mla_fwd(_ptr(q), _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd),
                                     _ptr(idx), idx.shape[1], float(scale), _ptr(out), _ptr(lse),
                                     _stream(stream)), "dsa_sparse_mla_fwd")
+    return out, lse
+
+
+def dsa_sparse_mla_workspace_size() -> int:
+    return int(lib().dsa_sparse_mla_workspace_size())
+
+
+def dsa_sparse_mla_fwd_ws(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale: float,
+                          workspace: Optional[torch.Tensor] = None,
+                          out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                          rows=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """dsa_sparse_mla_fwd with scratch for splitting the rows of a partly filled
+    last wave (include/dsa.h); ``workspace`` is any 256-B aligned device tensor
+    (a fresh one of dsa_sparse_mla_workspace_size() bytes when None)."""
+    T = q.shape[0]
+    if workspace is None:
+        workspace = torch.empty(dsa_sparse_mla_workspace_size(), dtype=torch.uint8,
+                                device=q.device)
+    if out is None:
+        out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().dsa_sparse_mla_fwd_ws(_ptr(q), _ptr(kv_cache), ctypes.byref(kvd),
+                                       ctypes.byref(qd), _ptr(idx), idx.shape[1], float(scale),
+                                       _ptr(workspace), nbytes, _ptr(out), _ptr(lse),
+                                       _stream(stream)), "dsa_sparse_mla_fwd_ws")
     return out, lse
 
 

@@ -75,9 +75,16 @@ def test_chunked_small_workspace_matches():
     assert small < need
     full = _gpu_forward(p)
     chunked = _gpu_forward(p, workspace_bytes=small)
-    np.testing.assert_array_equal(chunked[0], full[0])
-    np.testing.assert_array_equal(chunked[1], full[1])
-    np.testing.assert_array_equal(chunked[2], full[2])
+    np.testing.assert_array_equal(chunked[0], full[0])   # the selection, bit for bit
+    # The attention of the rows of a partly filled last wave is split into key
+    # segments when the workspace holds their partial outputs (the full one does,
+    # the small one does not): those rows agree up to rounding, the others exactly.
+    wave = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    n_whole = 1500 - 1500 % wave
+    np.testing.assert_array_equal(chunked[1][:n_whole], full[1][:n_whole])
+    np.testing.assert_array_equal(chunked[2][:n_whole], full[2][:n_whole])
+    assert np.abs(chunked[2] - full[2]).max() <= 5e-5
+    assert np.all(np.abs(chunked[1] - full[1]) <= 2.0 ** -7 * np.abs(chunked[1]) + 2e-3)
     rows = np.array([0, 5, 777, 1499])
     _check_forward(p, rows, workspace_bytes=small)
 
