@@ -259,32 +259,43 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
     bool overflow = false;
     float4 cur4[4], nxt4[4];
     load16(0, cur4);
+    // key >= tau_low <=> score >= thr (order-preserving keys, -0.0 == +0.0, no NaN)
+    const float thr = key_score(tau_low);
 #pragma unroll 1
     for (int base = 0; base < n; base += kStep) {
       if (base + kStep < n) load16(base + kStep, nxt4);
-      uint32_t kk[16];
+      const int e0 = base + 16 * tid;
+      uint32_t mask = 0;  // bit u: key e0 + u is kept
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        kk[4 * u] = score_key(cur4[u].x);
-        kk[4 * u + 1] = score_key(cur4[u].y);
-        kk[4 * u + 2] = score_key(cur4[u].z);
-        kk[4 * u + 3] = score_key(cur4[u].w);
+        mask |= (cur4[u].x >= thr ? 1u : 0u) << (4 * u);
+        mask |= (cur4[u].y >= thr ? 2u : 0u) << (4 * u);
+        mask |= (cur4[u].z >= thr ? 4u : 0u) << (4 * u);
+        mask |= (cur4[u].w >= thr ? 8u : 0u) << (4 * u);
       }
-      const int e0 = base + 16 * tid;
-      uint32_t c = 0;
-#pragma unroll
-      for (int u = 0; u < 16; ++u) c += (e0 + u < n) && kk[u] >= tau_low;
-      const uint32_t excl = block_exclusive_scan(c, misc, misc + 32);
+      if (base + kStep > n) {  // the last step: no key at or past n
+        const int left = n - e0;
+        mask &= left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u);
+      }
+      const uint32_t excl = block_exclusive_scan(__popc(mask), misc, misc + 32);
       const uint32_t tot = misc[32];
       uint32_t w = m_run + excl;
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        if ((e0 + u < n) && kk[u] >= tau_low) {
-          if (w < (uint32_t)kTopkCandCap) {
-            cand_key[w] = kk[u];
-            cand_pos[w] = e0 + u;
+      if (mask) {
+        auto put = [&](int u, float x) {
+          if ((mask >> u) & 1u) {
+            if (w < (uint32_t)kTopkCandCap) {
+              cand_key[w] = score_key(x);
+              cand_pos[w] = e0 + u;
+            }
+            ++w;
           }
-          ++w;
+        };
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          put(4 * u, cur4[u].x);
+          put(4 * u + 1, cur4[u].y);
+          put(4 * u + 2, cur4[u].z);
+          put(4 * u + 3, cur4[u].w);
         }
       }
       m_run += tot;
