@@ -190,7 +190,30 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const int64_t t = (int64_t)b * p.q_per_seq + qi;  // global query row
   const int d0 = 256 * (int)rank;        // first value dim (and first key dim) of this CTA
   const int r0 = 512 + 32 * (int)rank;   // this CTA's quarter of the rope dims
-  const int nblk = (e1 - e0 + kMlaBlk - 1) / kMlaBlk;
+  // Position of this query row and validity of its sequence.
+  const int seqlen = p.seqlens ? __ldg(p.seqlens + b) : p.max_ctx;
+  const bool seq_ok = seqlen >= p.q_per_seq && seqlen <= p.max_ctx;
+  const int pos = seqlen - p.q_per_seq + qi;
+  // Blocks after the last entry inside [0, pos] hold only masked keys and change
+  // nothing (no weight, no new maximum): the cluster stops at that entry's block
+  // (the top-k pads a row of fewer than k visible keys with -1 at its end). Only
+  // rows with fewer than k visible keys look (a uniform branch: both CTAs of the
+  // pair see the same row); the others run every block.
+  int nblk = (e1 - e0 + kMlaBlk - 1) / kMlaBlk;
+  if (seq_ok && pos + 1 < p.k) {
+    __shared__ int last_w[kMlaThreads / 32];
+    int last = -1;
+    for (int e = tid; e < e1 - e0; e += kMlaThreads) {
+      const int sel = __ldg(p.idx + t * p.k + e0 + e);
+      if (seq_ok && sel >= 0 && sel <= pos) last = e;
+    }
+    last = __reduce_max_sync(0xffffffffu, last);
+    if (lane == 0) last_w[warp] = last;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kMlaThreads / 32; ++i) last = max(last, last_w[i]);
+    nblk = max(1, (last + kMlaBlk) / kMlaBlk);  // one all-masked block when none is valid
+  }
 
   if (tid == 0) {
     for (int i = 0; i < kMlaStages; ++i) {
@@ -240,11 +263,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const uint64_t TO = p.timeout_ns;
   int drain_dummy = 0;
   volatile int* no_abort = &drain_dummy;
-
-  // Position of this query row and validity of its sequence.
-  const int seqlen = p.seqlens ? __ldg(p.seqlens + b) : p.max_ctx;
-  const bool seq_ok = seqlen >= p.q_per_seq && seqlen <= p.max_ctx;
-  const int pos = seqlen - p.q_per_seq + qi;
 
   if (warp == 1) {
     // ------------------------------------------------------------ row resolver

@@ -105,6 +105,27 @@ def test_dense_rows_equal_dense_causal_mqa():
     check_attention(o_g[rows], l_g[rows], o_r, l_r)
 
 
+@pytest.mark.parametrize("ws", [False, True])
+def test_short_rows_with_scattered_and_trailing_entries(ws):
+    """Rows with fewer than k visible keys stop after the block of their last entry
+    inside [0, pos]: entries scattered among -1 pads, a valid entry in the very last
+    slot, out-of-range entries after the last valid one, and a row whose only valid
+    entry comes first."""
+    p = synth.prefill(L=1500, seed=49)
+    rows = np.array([0, 1, 47, 48, 100, 700, 1499])
+    rng = np.random.default_rng(9)
+    idx = np.full((1500, 2048), -1, np.int32)
+    for t in range(1500):
+        n = t + 1
+        slots = np.sort(rng.choice(2048, n, replace=False))
+        idx[t, slots] = rng.permutation(n)          # every visible key once, scattered
+    idx[700, 2047] = 3                               # a valid entry in the last slot
+    idx[100, 1900:] = 5000                           # beyond pos after the last valid entry
+    idx[1] = -1
+    idx[1, 0] = 1                                    # only the first slot is valid
+    _check(p, idx, rows=rows, ws=ws)
+
+
 def test_empty_selection_gives_zero_and_neg_inf():
     p = synth.decode(batch=2, ctx=300, q_per_seq=1, seed=45)
     idx = np.full((2, 128), -1, np.int32)
