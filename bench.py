@@ -244,23 +244,35 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------------------
-def mla_split_launches(rows: int, k: int, scratch_bytes: int) -> int:
-    """Kernel launches of one dsa_sparse_mla_fwd_ws call: the attention, plus the
-    segment merge when the library's rule splits the rows of a last wave that is at
-    most half full (clusters of 2 SMs; 2..8 segments of >= 6 blocks of 48 keys, as
-    many as the scratch holds at 256.5 KB each). Used for the launch count only."""
-    wave = torch.cuda.get_device_properties(0).multi_processor_count // 2
+MLA_PART_BYTES = 128 * 512 * 4 + 128 * 4  # one segment's fp32 output and LSE
+
+
+def mla_split_plan(rows: int, k: int, scratch_bytes: int, sms=None):
+    """(split rows, segments per split row) of one dsa_sparse_mla_fwd_ws call under
+    the library's rule: the rows of a last wave (clusters of 2 SMs) that is at most
+    half full run as 2..8 segments of >= 6 blocks of 48 keys, as many as the scratch
+    holds. Used for the launch count; tests pin it to the library's workspace sizes."""
+    if sms is None:
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+    wave = sms // 2
     tail = rows % wave if wave >= 2 and rows > 0 else 0
     if tail == 0:
-        return 1
+        return 0, 1
     nb = -(-k // 48)
     s = min(wave // tail, 8, nb // 6)
-    while s >= 2 and tail * s * (128 * 512 * 4 + 128 * 4) > scratch_bytes:
+    while s >= 2 and tail * s * MLA_PART_BYTES > scratch_bytes:
         s -= 1
     if s < 2:
-        return 1
+        return 0, 1
     bps = -(-nb // s)
-    return 2 if -(-nb // bps) >= 2 else 1
+    nseg = -(-nb // bps)
+    return (tail, nseg) if nseg >= 2 else (0, 1)
+
+
+def mla_split_launches(rows: int, k: int, scratch_bytes: int) -> int:
+    """Kernel launches of one dsa_sparse_mla_fwd_ws call: the attention, plus the
+    segment merge when rows are split."""
+    return 2 if mla_split_plan(rows, k, scratch_bytes)[0] else 1
 
 
 class Runner:

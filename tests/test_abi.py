@@ -140,3 +140,28 @@ def test_workspace_size_plan(lib):
     assert n == 131072 * 2048 * 4 + 4096 * 131072 * 4
     # invalid geometry -> 0
     assert lib.dsa_workspace_size(by(kv), by(dsa.QDescC(5, 131072, 0, 0)), 2048) == 0
+
+
+@pytest.mark.parametrize("batch,q_per_seq,max_ctx,k", [
+    (4, 1, 4096, 2048),      # one partial wave: every row split (7 segments)
+    (40, 2, 512, 2048),      # 80 rows: a 6-row tail after one wave of 74
+    (1, 1500, 1500, 2048),   # prefill: 20-row tail, 3 segments
+    (3, 1, 300, 100),        # too few key blocks to split
+    (37, 2, 256, 2048),      # exactly one full wave: no split
+])
+def test_workspace_size_includes_the_split_rows(lib, batch, q_per_seq, max_ctx, k):
+    """Without a GPU the library plans for 148 SMs; the benchmark's mirror of the
+    split rule must give the same scratch the library reserves."""
+    from bench import MLA_PART_BYTES, mla_split_plan
+    from sparse_attention_05_b200 import dsa
+    by = ctypes.byref
+    kv, q = _kv(batch=batch, max_ctx=max_ctx), dsa.QDescC(batch * q_per_seq, q_per_seq, 0, 0)
+    n = lib.dsa_workspace_size(by(kv), by(q), k)
+    rows = batch * q_per_seq
+    idx = -(-rows * k * 4 // 256) * 256
+    ld = -(-max_ctx // 128) * 128
+    score = -(-min(q_per_seq, max(1, (2 << 30) // (ld * 4 * batch))) * batch * ld * 4 // 256) * 256
+    n_split, nseg = mla_split_plan(rows, k, 1 << 62, sms=148)
+    part = -(-n_split * nseg * MLA_PART_BYTES // 256) * 256
+    assert n == idx + max(score, part)
+    assert lib.dsa_sparse_mla_workspace_size() == 74 * MLA_PART_BYTES
