@@ -16,7 +16,7 @@ Sources (web pages on DeepSeek-V3.2-Exp, cited by page and section):
         128-d indexer key cache per token, 512-d latent key cache, the four-step
         flow (projections -> indexer scores -> top-k -> sparse MLA).
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 
 * Indexer score, [TR] §1 Eq. 1 (missing image; the prose names H^I heads,
   q^I_{t,j} in R^{d_I}, a scalar weight w^I_{t,j}, keys k^I_s, ReLU):
