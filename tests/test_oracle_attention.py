@@ -118,6 +118,27 @@ def test_permutation_and_padding_invariance():
     np.testing.assert_array_equal(l3, l1)
 
 
+def test_disjoint_parts_merge_to_the_whole_selection():
+    """Attention over a set equals the merge of attention over disjoint parts of it:
+    LSE = ln sum_s e^{LSE_s}, o = sum_s e^{LSE_s - LSE} o_s (an empty part has
+    LSE = -inf and weight 0). The split rows of the GPU path rely on this identity."""
+    p = synth.decode(batch=2, ctx=300, q_per_seq=1, seed=15, dims=synth.Dims(heads=4, topk=96))
+    a = oracle_args(p)
+    rng = np.random.default_rng(2)
+    idx = np.stack([rng.choice(int(a["q_pos"][t]) + 1, 96, replace=False)
+                    for t in range(p.num_q)]).astype(np.int32)
+    o, l = sparse_mla(a["q"], a["kv"], a["q_seq"], a["q_pos"], idx, p.scale, 512)
+    parts = [idx[:, :40], idx[:, 40:41], np.full((p.num_q, 5), -1, np.int32), idx[:, 41:]]
+    res = [sparse_mla(a["q"], a["kv"], a["q_seq"], a["q_pos"], x, p.scale, 512) for x in parts]
+    ls = np.stack([r[1] for r in res])                       # [parts, T, H]
+    lse = np.logaddexp.reduce(ls, axis=0)
+    wts = np.exp(ls - lse[None])                             # empty part: exp(-inf) = 0
+    om = sum(w[..., None] * r[0] for w, r in zip(wts, res))
+    np.testing.assert_allclose(lse, l, rtol=1e-13, atol=1e-12)
+    np.testing.assert_allclose(om, o, rtol=1e-11, atol=1e-12)
+    assert np.all(np.isneginf(ls[2]))
+
+
 def test_empty_selection():
     o, lse = sparse_mla_token(np.ones((2, 8)), [], 1.0, 4)
     assert np.all(o == 0) and np.all(np.isneginf(lse))
