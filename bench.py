@@ -704,6 +704,20 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
+def host_cpu() -> dict:
+    """The host the oracle ran on: CPU model and logical core count."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count() or 1}
+
+
 def cpu_baseline(p: synth.Problem, name: str, budget_s: float = 12.0, seed: int = 0,
                  mha=None) -> dict:
     """The oracle on a bounded sample: two query rows of a random sequence per call
@@ -728,7 +742,8 @@ def cpu_baseline(p: synth.Problem, name: str, budget_s: float = 12.0, seed: int 
         seqs.append(b)
     what = ("indexer+top-k (rows past k)+masked MHA per row" if mha is not None
             else "full indexer+top-k+attention per row")
-    return {"value": rows_done / elapsed, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    return {"value": rows_done / elapsed, "unit": UNIT, "cores": blas_threads(), **host_cpu(),
+            "kind": "oracle",
             "sample": f"{rows_done} query rows of {name} (sequences {seqs[:8]}"
                       f"{'...' if len(seqs) > 8 else ''}), {what}, "
                       f"{elapsed:.1f} s of host time"}
@@ -770,7 +785,7 @@ def reference_arm(args):
             "config": {"workload": args.workload, **WORKLOADS[args.workload],
                        **({"mode": "mha (masked MHA emulation of DSA)"} if m is not None else {}),
                        "sample_rows_per_step": per_step_rows},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), **host_cpu(),
                              "kind": "oracle",
                              "sample": f"{per_step_rows} query rows of one random sequence per "
                                        f"step, {args.steps} steps"},
