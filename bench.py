@@ -171,10 +171,57 @@ def roofline(kernel: str, work: dict, avg_s: float, peaks: dict, long_step: bool
         peak = peaks["hbm_gbs"]
         r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s"}
     r["frac"] = achieved / peak
+    if r["unit"] == "TFLOP/s" and w["flop_dtype"] == "fp8" and peaks.get("fp8_tflops"):
+        r["frac_of_measured_fp8"] = achieved / peaks["fp8_tflops"]
     r["peak_source"] = peaks["source"] + ("" if r["unit"] == "GB/s" else
                                           (" sustained" if long_step else " burst") +
                                           (" x2 (fp8 from bf16)" if w["flop_dtype"] == "fp8" else ""))
     return r
+
+
+def step_roofline(work: dict, kernels, step_s: float, peaks: dict, long_step: bool) -> dict:
+    """Roofline of the whole step: T_roof = max(all bytes / HBM, FP8 FLOP / FP8 peak +
+    BF16 FLOP / BF16 peak) over the step's kernels, against the measured step time."""
+    bf16 = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
+    tflops = {"bf16": bf16, "fp8": 2.0 * bf16}
+    nbytes = sum(work[k]["bytes"] for k in kernels)
+    t_mem = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_cmp = sum(work[k]["flop"] / (tflops[work[k]["flop_dtype"]] * 1e12)
+                for k in kernels if work[k]["flop"])
+    t_roof = max(t_mem, t_cmp)
+    return {"bound": "tensor" if t_cmp > t_mem else "hbm", "roofline_ms": 1e3 * t_roof,
+            "ms_per_step": 1e3 * step_s, "frac": t_roof / step_s,
+            "hbm_ms": 1e3 * t_mem, "tensor_ms": 1e3 * t_cmp, "bytes": nbytes,
+            "kernels": list(kernels)}
+
+
+def measure_fp8_peak() -> dict:
+    """Dense FP8 (E4M3 x E4M3 -> bf16) throughput of cuBLASLt through torch._scaled_mm,
+    8192^3, best of 10 bursts of 10: the measured FP8 figure that sits next to the
+    2 x BF16 denominator (context, not the product path)."""
+    n = 8192
+    try:
+        a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device="cuda")
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(10):
+                torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1) / 1e3 / 10)
+        del a, b
+        torch.cuda.empty_cache()
+        return {"fp8_tflops": 2 * n ** 3 / best / 1e12,
+                "fp8_source": "torch._scaled_mm e4m3 x e4m3 -> bf16, 8192^3, best of 10 "
+                              "bursts of 10, measured in this run (cuBLASLt)"}
+    except Exception as e:  # noqa: BLE001 - context only
+        return {"fp8_tflops": None, "fp8_source": f"not measured: {type(e).__name__}"}
 
 
 def dram_traffic(kernel: str, workload: str):
@@ -742,11 +789,14 @@ def cpu_baseline(p: synth.Problem, name: str, budget_s: float = 12.0, seed: int 
         seqs.append(b)
     what = ("indexer+top-k (rows past k)+masked MHA per row" if mha is not None
             else "full indexer+top-k+attention per row")
-    return {"value": rows_done / elapsed, "unit": UNIT, "cores": blas_threads(), **host_cpu(),
+    nt = blas_threads()
+    return {"value": rows_done / elapsed, "unit": UNIT, "cores": nt, "processes": 1,
+            "parallelism": f"1 process; numpy's BLAS on {nt} threads (matmuls), the rest "
+                           f"single-threaded", **host_cpu(),
             "kind": "oracle",
             "sample": f"{rows_done} query rows of {name} (sequences {seqs[:8]}"
                       f"{'...' if len(seqs) > 8 else ''}), {what}, "
-                      f"{elapsed:.1f} s of host time"}
+                      f"{elapsed:.1f} s of host time, 1 process with {nt} BLAS threads"}
 
 
 def reference_arm(args):
@@ -785,10 +835,11 @@ def reference_arm(args):
             "config": {"workload": args.workload, **WORKLOADS[args.workload],
                        **({"mode": "mha (masked MHA emulation of DSA)"} if m is not None else {}),
                        "sample_rows_per_step": per_step_rows},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), **host_cpu(),
-                             "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "processes": 1, **host_cpu(), "kind": "oracle",
                              "sample": f"{per_step_rows} query rows of one random sequence per "
-                                       f"step, {args.steps} steps"},
+                                       f"step, {args.steps} steps, 1 process with "
+                                       f"{blas_threads()} BLAS threads"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -796,6 +847,79 @@ def reference_arm(args):
 
 
 # ----------------------------------------------------------------------------------------
+def measure(r, work: dict, workload: str, steps: int, warmup: int, world: int, local: int,
+            soak_s: float, ev_names, peaks: dict) -> dict:
+    """Warm-up, a short untimed soak (clock samples start), then exactly ``steps``
+    steps bracketed by a barrier and a device synchronize on both sides, timed with
+    CUDA events on the launching stream (max over ranks); per-kernel CUDA events
+    inside the same region give each stage's time and roofline."""
+    for _ in range(warmup):
+        r.step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < soak_s:
+        r.step()
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = {n: [] for n in ev_names}
+    start = _record()
+    for _ in range(steps):
+        r.step(ev)
+    stop = _record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    secs = max_over_ranks(start.elapsed_time(stop) / 1e3, world)
+
+    per_kernel = {kname: _pairs_ms(e) for kname, e in ev.items() if e}
+    launches = {kname: len(v) for kname, v in per_kernel.items()}
+    total_ms = {kname: sum(v) for kname, v in per_kernel.items()}
+    # the dominant kernel (the all-gather of the context-parallel mode is a collective)
+    dominant = max((k for k in total_ms if k != "allgather"), key=total_ms.get)
+    long_step = secs / steps > 0.05
+    avg_s = total_ms[dominant] / 1e3 / steps  # one step's worth of that kernel
+    roof = roofline(dominant, work, avg_s, peaks, long_step)
+    roof["kernel"] = dominant
+    roof["launches_per_step"] = launches[dominant] // steps
+    roof["traffic"] = dram_traffic(dominant, workload)
+    roof["step"] = step_roofline(work, [k for k in per_kernel if k != "allgather"],
+                                 secs / steps, peaks, long_step)
+    stages = {}
+    for kname in per_kernel:
+        a = total_ms[kname] / 1e3 / steps
+        rf = roofline(kname, work, a, peaks, long_step)
+        stages[kname] = {"ms_per_step": 1e3 * a, "share": total_ms[kname] / sum(total_ms.values()),
+                         "bound": rf["bound"], "frac": rf["frac"],
+                         "achieved": rf["achieved"], "unit": rf["unit"]}
+        if "frac_of_measured_fp8" in rf:
+            stages[kname]["frac_of_measured_fp8"] = rf["frac_of_measured_fp8"]
+    return {"secs": secs, "clocks": clk, "roofline": roof, "stages": stages,
+            "launches": launches}
+
+
+def secondary_prefill(args, world: int, local: int, rank: int, peaks: dict) -> dict:
+    """The metric's other half: the 128K causal prefill step (MQA mode) measured in the
+    same run as the decode line, with the same protocol (3 warm-up, 3 timed steps)."""
+    name = "prefill_128k"
+    p = make_problem(name, "cuda", seed_offset=rank)
+    r = Runner(p)
+    work = algorithmic_work(p)
+    steps, warmup = 3, 3
+    m = measure(r, work, name, steps, warmup, world, local, 0.0,
+                ("indexer", "topk", "sparse_mla"), peaks)
+    out = {"workload": name, **WORKLOADS[name], "value": world * p.num_q * steps / m["secs"],
+           "unit": UNIT, "ms_per_step": 1e3 * m["secs"] / steps, "steps": steps,
+           "warmup": warmup, "roofline": m["roofline"], "stages": m["stages"],
+           "clocks": m["clocks"], "gpu_launches": r.launches_per_step * steps,
+           "query_rows_per_gpu": p.num_q}
+    del r, p
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -816,6 +940,10 @@ def main(argv=None):
                     help="fused indexer -> top-k selection (no stored score rows)")
     ap.add_argument("--mode", default="mqa", choices=["mqa", "mha"],
                     help="mha: short-prefill DSA in MLA's MHA mode (masked MHA; prefill_8k)")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the 128K prefill half of the metric in the default run")
+    ap.add_argument("--no-fp8-peak", action="store_true",
+                    help="skip the live FP8 GEMM measurement (context for the FP8 fractions)")
     ap.add_argument("--soak-s", type=float, default=1.0,
                     help="untimed seconds of steps right before the timed region (clock samples)")
     args = ap.parse_args(argv)
@@ -859,54 +987,22 @@ def main(argv=None):
         work = algorithmic_work(p)
     peaks = load_peaks()
 
-    for _ in range(args.warmup):
-        r.step()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local)
-    t_soak = time.perf_counter()
-    while time.perf_counter() - t_soak < args.soak_s:
-        r.step()
-        torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
     if args.mode == "mha":
-        ev = {n: [] for n in MhaRunner.STAGES}
+        ev_names = MhaRunner.STAGES
     elif args.cp:
-        ev = {"allgather": [], "indexer": [], "topk": [], "sparse_mla": []}
+        ev_names = ("allgather", "indexer", "topk", "sparse_mla")
     elif args.fused:
-        ev = {"select_fused": [], "sparse_mla": []}
+        ev_names = ("select_fused", "sparse_mla")
     else:
-        ev = {"indexer": [], "topk": [], "sparse_mla": []}
+        ev_names = ("indexer", "topk", "sparse_mla")
     if args.kl:
-        ev["indexer_kl"] = []
-    start = _record()
-    for _ in range(args.steps):
-        r.step(ev)
-    stop = _record()
-    torch.cuda.synchronize()
-    barrier(world)
-    clk = clocks.stop()
-    secs_local = start.elapsed_time(stop) / 1e3
-    secs = max_over_ranks(secs_local, world)
-
-    per_kernel = {kname: _pairs_ms(e) for kname, e in ev.items() if e}
-    launches = {kname: len(v) for kname, v in per_kernel.items()}
-    total_ms = {kname: sum(v) for kname, v in per_kernel.items()}
-    # the dominant kernel (the all-gather of the context-parallel mode is a collective)
-    dominant = max((k for k in total_ms if k != "allgather"), key=total_ms.get)
-    long_step = secs / args.steps > 0.05
-    avg_s = total_ms[dominant] / 1e3 / args.steps  # one step's worth of that kernel
-    roof = roofline(dominant, work, avg_s, peaks, long_step)
-    roof["kernel"] = dominant
-    roof["launches_per_step"] = launches[dominant] // args.steps
-    roof["traffic"] = dram_traffic(dominant, args.workload)
-    stages = {}
-    for kname in per_kernel:
-        a = total_ms[kname] / 1e3 / args.steps
-        rf = roofline(kname, work, a, peaks, long_step)
-        stages[kname] = {"ms_per_step": 1e3 * a, "share": total_ms[kname] / sum(total_ms.values()),
-                         "bound": rf["bound"], "frac": rf["frac"],
-                         "achieved": rf["achieved"], "unit": rf["unit"]}
+        ev_names = ev_names + ("indexer_kl",)
+    peaks["fp8_tflops"] = None
+    if not args.no_fp8_peak:
+        peaks.update(measure_fp8_peak())
+    m = measure(r, work, args.workload, args.steps, args.warmup, world, local, args.soak_s,
+                ev_names, peaks)
+    secs, clk, roof, stages = m["secs"], m["clocks"], m["roofline"], m["stages"]
 
     # context parallel: the end-to-end arm of the public call is the single-GPU one
     e2e = None if (args.no_e2e or args.cp or args.fused) else \
@@ -914,6 +1010,20 @@ def main(argv=None):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(p, args.workload, mha=r.m if args.mode == "mha" else None)
+
+    # the metric's other half, measured in the same run: the default (decode) line
+    # also carries the 128K prefill step
+    secondary = None
+    run_secondary = (args.workload == DEFAULT_WORKLOAD and not args.no_secondary and
+                     not (args.cp or args.fused or args.kl or args.batch) and args.mode == "mqa")
+    n_launch = r.launches_per_step * args.steps
+    rows_primary = len(r.rows) if args.cp else p.num_q
+    rows_problem = p.num_q
+    if run_secondary:
+        del r, p
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        secondary = secondary_prefill(args, world, local, rank, peaks)
 
     if rank == 0:
         cfg = {"workload": args.workload, **WORKLOADS[args.workload],
@@ -924,13 +1034,13 @@ def main(argv=None):
                    "d_v": 128, "d_latent": 576} if args.mode == "mha" else
                   {"heads": 128, "d_qk": 576, "d_v": 512}),
                "h_idx": 64, "d_idx": 128,
-               "query_rows_per_gpu": len(r.rows) if args.cp else p.num_q,
+               "query_rows_per_gpu": rows_primary,
                "l2": "inputs larger than L2 (no flush)",
                "parallelism": (f"cp{world} (caches sharded by token and all-gathered every "
                                f"step, query rows zigzag across GPUs)" if args.cp else
                                f"dp{world} (independent sequences per GPU)")}
         # context parallel: the job processes one sequence's L rows per step
-        rows_job = p.num_q if args.cp else world * p.num_q
+        rows_job = rows_problem if args.cp else world * rows_problem
         line = {
             "metric": METRIC, "value": rows_job * args.steps / secs,
             "unit": UNIT,
@@ -941,9 +1051,11 @@ def main(argv=None):
             "roofline": roof, "stages": stages, "clocks": clk,
             # our kernels launched in the timed region (the fused selection's event
             # pair spans its four launches per chunk of rows)
-            "gpu_launches": r.launches_per_step * args.steps,
+            "gpu_launches": n_launch,
             "e2e": e2e, "cpu_baseline": cpu, "peaks": peaks,
         }
+        if secondary is not None:
+            line["secondary"] = secondary
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

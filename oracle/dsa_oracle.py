@@ -194,17 +194,28 @@ def indexer_scores(q_idx, w, k_idx, k_scale, q_seq, q_pos, *, ld, rows=None,
     else:
         q_hat = np.asarray(q_idx, np.float64)
         head_w = np.asarray(w, np.float64)
+    # a sequence's visible keys are resolved and decoded once for a run of its rows,
+    # up to the last position those rows see (decoding is elementwise: the same values
+    # as decoding each row's keys separately); one sequence is held at a time
+    n_seq = {}
+    for t in rows:
+        b = int(q_seq[t])
+        n_seq[b] = max(n_seq.get(b, 0), int(q_pos[t]) + 1)
+    held_b, held = None, None
     for r, t in enumerate(rows):
         b = int(q_seq[t])
         n = int(q_pos[t]) + 1
-        pos = np.arange(n)
-        keys = resolve_kv_rows(k_idx, b, pos, block_table, page_size)
-        if fp8:
-            k_hat = e4m3_decode(keys)
-            s_k = resolve_kv_rows(k_scale, b, pos, block_table, page_size).astype(np.float64)
-        else:
-            k_hat = np.asarray(keys, np.float64)
-            s_k = np.ones(n)
+        if b != held_b:
+            pos_b = np.arange(n_seq[b])
+            keys = resolve_kv_rows(k_idx, b, pos_b, block_table, page_size)
+            if fp8:  # all 256 codes decoded once, then looked up (the same values)
+                held = (e4m3_decode(np.arange(256, dtype=np.uint8))[np.asarray(keys, np.uint8)],
+                        resolve_kv_rows(k_scale, b, pos_b, block_table,
+                                        page_size).astype(np.float64))
+            else:
+                held = (np.asarray(keys, np.float64), np.ones(n_seq[b]))
+            held_b = b
+        k_hat, s_k = held[0][:n], held[1][:n]
         dots = q_hat[t] @ k_hat.T  # [H^I, n]
         score = s_k * (head_w[t] @ np.maximum(dots, 0.0))
         out[r, :n] = score.astype(np.float32)

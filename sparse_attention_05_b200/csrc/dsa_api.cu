@@ -79,25 +79,56 @@ dsa_status_t check_geometry(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, Geom
   return DSA_OK;
 }
 
+// Per-device state: kernel attributes belong to each device's context, so a
+// process that drives several GPUs sets them (and reads the SM count) on each.
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
 int num_sms() {
-  static int sms = [] {
-    int dev = 0, n = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
-  }();
-  return sms;
+  static std::atomic<int> sms[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  int n = sms[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 2)
+      n = 148;
+    sms[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+// Runs `fn` (which returns a cudaError_t) once per device and remembers its result.
+struct DeviceOnce {
+  std::mutex mu;
+  bool done[kMaxDevices] = {};
+  cudaError_t err[kMaxDevices] = {};
+};
+
+template <typename Fn>
+cudaError_t once_per_device(DeviceOnce& o, Fn&& fn) {
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(o.mu);
+  if (!o.done[dev]) {
+    o.err[dev] = fn();
+    o.done[dev] = true;
+  }
+  return o.err[dev];
 }
 
 // ---- top-k launch ------------------------------------------------------------------
 dsa_status_t launch_topk(const float* scores, int64_t ld, const Geometry& g, int row_begin,
                          int row_count, int k, int32_t* idx, cudaStream_t stream,
                          int tile_stride = 1, float* kth_out = nullptr) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kTopkSmemBytes);
+  static DeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [] {
+    return cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kTopkSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   TopkParams p{scores, ld, g.seqlens, g.max_ctx, g.q_per_seq, row_begin, row_count, g.batch, k,
@@ -152,14 +183,14 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
                             const float* k_scale, const Geometry& g, float* scores, int64_t ld,
                             int row_begin, int row_count, cudaStream_t stream,
                             int tile_stride = 1, const IdxFilter& filt = IdxFilter()) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(indexer_kernel<false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmemBytes);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(indexer_kernel<true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmemBytes);
+  static DeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [] {
+    cudaError_t e = cudaFuncSetAttribute(indexer_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(indexer_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kIdxSmemBytes);
+    return e;
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   CUtensorMap tm;
@@ -242,11 +273,10 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
                                const int32_t* idx, int k, float scale, void* out, float* lse,
                                cudaStream_t stream, void* scratch = nullptr,
                                size_t scratch_bytes = 0) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(sparse_mla_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmemBytes);
+  static DeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [] {
+    return cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kMlaSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   // the latent cache as [cache_rows][576] bf16, gathered 64 dims of one row per box row
@@ -318,11 +348,10 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
 dsa_status_t launch_indexer_kl(const void* q, const void* kv_cache, const Geometry& g,
                                const int32_t* idx, int k, float scale, const float* lse,
                                const float* scores, int64_t ld, float* kl, cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(indexer_kl_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kKlSmemBytes);
+  static DeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [] {
+    return cudaFuncSetAttribute(indexer_kl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kKlSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   KlParams p{};
@@ -425,11 +454,10 @@ bool mha_fits(const Geometry& g, int64_t ctx_pad) {
 dsa_status_t launch_up_proj(const void* kv_cache, const void* w_uk, const void* w_uv,
                             const Geometry& g, void* k_nope, void* k_rope, void* v,
                             int64_t ctx_pad, cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(mla_up_proj_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kUpSmemBytes);
+  static DeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [] {
+    return cudaFuncSetAttribute(mla_up_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kUpSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   CUtensorMap tm_lat, tm_uk, tm_uv;
@@ -470,11 +498,10 @@ dsa_status_t launch_selection_mask(const int32_t* idx, int k, const Geometry& g,
                                    cudaStream_t stream) {
   const size_t smem = (size_t)mask_ld * 4;
   if (smem > 227 * 1024) return DSA_ERR_UNSUPPORTED_SHAPE;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(selection_mask_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  static DeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [] {
+    return cudaFuncSetAttribute(selection_mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                227 * 1024);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   MaskParams p{idx, g.seqlens, mask, mask_ld, k, g.batch, g.max_ctx, g.q_per_seq, row_begin,
@@ -489,11 +516,10 @@ dsa_status_t launch_masked_mha(const void* q_mha, const void* k_nope, const void
                                const void* v, int64_t ctx_pad, const Geometry& g,
                                const uint32_t* mask, int64_t mask_ld, int k, float scale,
                                void* out, float* lse, cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(masked_mha_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kFaSmemBytes);
+  static DeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [] {
+    return cudaFuncSetAttribute(masked_mha_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kFaSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   CUtensorMap tm_q, tm_kn, tm_kr, tm_v;
@@ -540,11 +566,10 @@ dsa_status_t launch_cand_select(const Geometry& g, int row_begin, int row_count,
                                 int32_t* idx, const uint32_t* ckey, const int32_t* cpos,
                                 const uint32_t* cnt, int cap, int32_t* redo_rows,
                                 uint32_t* redo_cnt, cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(cand_select_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kCandSmemBytes);
+  static DeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [] {
+    return cudaFuncSetAttribute(cand_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kCandSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   CandParams p{ckey, cpos, cnt, cap, g.seqlens, g.max_ctx, g.q_per_seq, row_begin, row_count,
@@ -627,10 +652,11 @@ dsa_status_t select_fused_chunk(const void* q_idx, const float* w, const void* k
       cudaStreamSynchronize(s) != cudaSuccess)
     return DSA_ERR_CUDA;
   if (n_redo == 0) return DSA_OK;
-  n_redo = std::min<uint32_t>(n_redo, (uint32_t)nrow);
+  n_redo = std::min<uint32_t>(n_redo, (uint32_t)nrow);  // the kernel never lists more
   std::vector<int32_t> rows(n_redo);
-  if (cudaMemcpy(rows.data(), redo_rows, (size_t)n_redo * 4, cudaMemcpyDeviceToHost) !=
-      cudaSuccess)
+  if (cudaMemcpyAsync(rows.data(), redo_rows, (size_t)n_redo * 4, cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
     return DSA_ERR_CUDA;
   std::vector<char> done(rc, 0);  // a window row index covers that row of every sequence
   for (int32_t wr : rows) {
@@ -651,7 +677,6 @@ dsa_status_t select_fused_chunk(const void* q_idx, const float* w, const void* k
 constexpr size_t kStaticScratchBytes = size_t(128) << 20;
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
 

@@ -416,7 +416,10 @@ __global__ void __launch_bounds__(kCandThreads, 2) cand_select_kernel(CandParams
   }
   const uint32_t m = p.cand_cnt[wrow];
   if (m < (uint32_t)p.k || m > (uint32_t)p.cand_cap) {
-    if (tid == 0) p.redo_rows[atomicAdd(p.redo_cnt, 1u)] = (int32_t)wrow;
+    if (tid == 0) {  // one entry per row at most, so the slot stays below the row count
+      const uint32_t slot = atomicAdd(p.redo_cnt, 1u);
+      if (slot < (uint32_t)p.batch * (uint32_t)p.row_count) p.redo_rows[slot] = (int32_t)wrow;
+    }
     return;
   }
   const int words = (n + 31) >> 5;  // <= kCandMaxWords (checked on the host)
