@@ -25,10 +25,14 @@
  *    H = 128 query heads, D = 576, D_v = 512, 1 <= k <= 2048, page size a
  *    multiple of 64. Anything else returns DSA_ERR_UNSUPPORTED_SHAPE; there is
  *    no fallback path.
- *  - Query geometry: query row t belongs to sequence b = t / q_per_seq and sits
- *    at position pos(t) = seqlen[b] - q_per_seq + (t % q_per_seq): the rows of a
- *    sequence are its last q_per_seq tokens (decode: 1 or 2; prefill: all L).
- *    Row t sees keys s in [0, pos(t)].
+ *  - Query geometry: the query rows of sequence b are its last q_len[b] tokens
+ *    (decode: the 1 or 2 newest; prefill: the whole prompt; chunked prefill: the
+ *    chunk just appended to a cache that already holds the earlier tokens). Row i
+ *    of sequence b (0 <= i < q_len[b]) is global query row t = t0[b] + i at
+ *    position pos(t) = seqlen[b] - q_len[b] + i, and sees keys s in [0, pos(t)].
+ *    Uniform batch (dsa_q_desc_t.q_start == NULL): q_len[b] = q_per_seq and
+ *    t0[b] = b * q_per_seq. Ragged batch: t0[b] = q_start[b] and
+ *    q_len[b] = q_start[b + 1] - q_start[b] (see dsa_q_desc_t).
  *  - Thread safety: calls may be issued from several host threads; calls
  *    that overlap on the GPU share only the device error word.
  */
@@ -82,15 +86,31 @@ typedef struct {
 
 /* Query rows. Each call processes the window of rows i in [row_begin,
  * row_begin + row_count) of every sequence (row_count = 0 means all rows from
- * row_begin on); rows outside the window are neither read nor written. Score
- * rows are stored compactly per window: window row i of sequence b is score
- * row b * row_count + (i - row_begin). Indices, queries, outputs and LSE keep
- * their global row t = b * q_per_seq + i. */
+ * row_begin through q_per_seq - 1); rows outside the window, and window rows a
+ * sequence of a ragged batch does not have (i >= q_len[b]), are neither read nor
+ * written. Score rows are stored compactly per window: window row i of sequence
+ * b is score row b * row_count + (i - row_begin), whether or not the sequence
+ * has that row. Indices, queries, outputs and LSE keep their global row
+ * t = t0[b] + i.
+ *
+ * Ragged batches (q_start != NULL; the varlen layout of a batch of prompts of
+ * different lengths, or of chunked-prefill pieces of different sizes, on one
+ * cache, "dynamic KV cache" in the DSA principle section of the nsmao.com
+ * report): sequence b owns the global rows [q_start[b], q_start[b + 1]), its
+ * last q_len[b] = q_start[b + 1] - q_start[b] tokens (0 allowed). q_start is
+ * device int32 [batch + 1], nondecreasing, q_start[0] >= 0, q_start[batch] <=
+ * num_q, every q_len[b] <= q_per_seq and <= seqlen[b]; the kernels check these
+ * and report DSA_ERR_BOUNDS through dsa_get_device_error for a sequence that
+ * breaks them (its rows are then skipped). The host cannot read q_start, so
+ * grids and score rows are sized for q_per_seq rows per sequence: choose it as
+ * the largest q_len. */
 typedef struct {
-  int32_t num_q;               /* T = batch * q_per_seq                                 */
-  int32_t q_per_seq;           /* query rows per sequence (>= 1)                        */
+  int32_t num_q;               /* T: batch * q_per_seq (uniform), rows in q_start's
+                                  range (ragged; at most batch * q_per_seq)             */
+  int32_t q_per_seq;           /* query rows per sequence (>= 1); ragged: the largest  */
   int32_t row_begin;           /* first row of the window (0 = from the first row)      */
-  int32_t row_count;           /* rows in the window (0 = through the last row)         */
+  int32_t row_count;           /* rows in the window (0 = through row q_per_seq - 1)    */
+  const int32_t* q_start;      /* NULL (uniform), or device int32 [batch + 1] (ragged)  */
 } dsa_q_desc_t;
 
 /* Lightning-indexer scores (Eq. 1 of the report, FP8 as its §1 allows).
@@ -171,6 +191,7 @@ DSA_API size_t dsa_sparse_mla_workspace_size(void);
  *  scores fp32 [batch * row_count][ld] indexer score rows of the window (as
  *         dsa_indexer_scores writes them); ld >= max_ctx
  *  kl     fp32 [batch * row_count] out, one term per row of the window.
+ * A window row a ragged batch's sequence does not have gets kl = 0.
  * Shapes: 128 heads x 576-d latents only. */
 DSA_API dsa_status_t dsa_indexer_kl(const void* q, const void* kv_cache, const dsa_kv_desc_t* kv,
                                     const dsa_q_desc_t* qd, const int32_t* idx, int32_t k,
@@ -325,8 +346,8 @@ DSA_API dsa_status_t dsa_masked_mha(const void* q_mha, const void* k_nope, const
 DSA_API size_t dsa_mha_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k);
 
 /* Short-prefill DSA in MHA mode: indexer scores and top-k for the rows with more
- * than k visible keys (when seqlens is NULL the rows with pos(t) + 1 <= k are
- * skipped; with a seqlens array every row of the window is scored), their
+ * than k visible keys (when seqlens and q_start are NULL the rows with pos(t) + 1
+ * <= k are skipped; otherwise every row of the window is scored), their
  * selection masks, the up-projection of the latent cache, then the masked MHA.
  * Inputs as for dsa_forward plus q_mha, w_uk and w_uv; out and lse as for
  * dsa_masked_mha. `workspace` (256-byte aligned) holds the indices (unless idx_out

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdsa.so")
 SOURCES = ["dsa_api.cu"]
-HEADERS = ["ptx.cuh", "topk.cuh", "indexer.cuh", "sparse_mla.cuh", "indexer_kl.cuh",
+HEADERS = ["ptx.cuh", "rows.cuh", "topk.cuh", "indexer.cuh", "sparse_mla.cuh", "indexer_kl.cuh",
            "mha_prefill.cuh"]
 
 NVCC_FLAGS = [
@@ -39,10 +39,10 @@ KERNEL_HEADER = {"indexer": "indexer.cuh", "topk": "topk.cuh", "sparse_mla": "sp
 
 def source_digest(kernel=None) -> str:
     """Digest of the CUDA sources and the ABI header (identifies a library build);
-    with ``kernel``, of that kernel's header and the shared PTX helpers only."""
+    with ``kernel``, of that kernel's header and the shared PTX and row helpers only."""
     import hashlib
     h = hashlib.sha256()
-    files = (["ptx.cuh", KERNEL_HEADER[kernel]] if kernel else SOURCES + HEADERS)
+    files = (["ptx.cuh", "rows.cuh", KERNEL_HEADER[kernel]] if kernel else SOURCES + HEADERS)
     for f in files:
         h.update(open(os.path.join(CSRC, f), "rb").read())
     if not kernel:

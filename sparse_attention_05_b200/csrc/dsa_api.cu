@@ -38,13 +38,19 @@ struct Geometry {
   int row_begin, row_count;  // window of rows per sequence
   const int32_t* block_table;
   const int32_t* seqlens;
+  const int32_t* q_start;    // ragged query rows ([batch + 1], device) or nullptr
   int64_t cache_rows;  // rows of each per-token cache array
 };
 
 dsa_status_t check_geometry(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, Geometry* g) {
   if (!kv || !q) return DSA_ERR_INVALID_ARG;
   if (kv->batch < 1 || kv->max_ctx < 1 || q->q_per_seq < 1) return DSA_ERR_INVALID_ARG;
-  if ((int64_t)kv->batch * q->q_per_seq != q->num_q) return DSA_ERR_INVALID_ARG;
+  if (q->q_start) {  // ragged: every sequence has at most q_per_seq rows
+    if (q->num_q < 0 || (int64_t)q->num_q > (int64_t)kv->batch * q->q_per_seq)
+      return DSA_ERR_INVALID_ARG;
+  } else if ((int64_t)kv->batch * q->q_per_seq != q->num_q) {
+    return DSA_ERR_INVALID_ARG;
+  }
   if (q->q_per_seq > kv->max_ctx) return DSA_ERR_INVALID_ARG;
   if (q->row_begin < 0 || q->row_begin >= q->q_per_seq || q->row_count < 0 ||
       q->row_count > q->q_per_seq - q->row_begin)
@@ -56,6 +62,7 @@ dsa_status_t check_geometry(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, Geom
   g->max_ctx = kv->max_ctx;
   g->q_per_seq = q->q_per_seq;
   g->num_q = q->num_q;
+  g->q_start = q->q_start;
   g->seqlens = kv->seqlens;
   g->block_table = nullptr;
   g->page_size = 0;
@@ -132,7 +139,7 @@ dsa_status_t launch_topk(const float* scores, int64_t ld, const Geometry& g, int
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   TopkParams p{scores, ld, g.seqlens, g.max_ctx, g.q_per_seq, row_begin, row_count, g.batch, k,
-               idx, tile_stride, kth_out};
+               idx, tile_stride, kth_out, g.q_start, g.num_q};
   const int64_t grid = (int64_t)g.batch * row_count;
   if (grid == 0) return DSA_OK;
   topk_kernel<<<(unsigned)grid, kTopkThreads, kTopkSmemBytes, stream>>>(p);
@@ -223,6 +230,8 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   p.cand_pos = filt.cand_pos;
   p.cand_cnt = filt.cand_cnt;
   p.cand_cap = filt.cand_cap;
+  p.q_start = g.q_start;
+  p.num_q = g.num_q;
   p.timeout_ns = g_timeout_ns.load();
   // every CTA takes an equal share of all key tiles (at most one CTA per tile)
   const int64_t max_tiles = (int64_t)p.num_groups * ((g.max_ctx + kIdxTile - 1) / kIdxTile);
@@ -305,6 +314,8 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
   p.row_count = g.row_count;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns.load();
+  p.q_start = g.q_start;
+  p.num_q = g.num_q;
   const int64_t rows = (int64_t)g.batch * g.row_count;
   if (rows == 0) return DSA_OK;
   const MlaSplit sp = plan_mla_split(rows, k, scratch ? scratch_bytes : 0);
@@ -340,6 +351,10 @@ dsa_status_t launch_sparse_mla(const void* q, const void* kv_cache, const Geomet
   c.row_begin = g.row_begin;
   c.row_count = g.row_count;
   c.q_per_seq = g.q_per_seq;
+  c.q_start = g.q_start;
+  c.seqlens = g.seqlens;
+  c.num_q = g.num_q;
+  c.max_ctx = g.max_ctx;
   mla_combine_kernel<<<dim3((unsigned)sp.n_split, kMlaHeads / 8), 256, 0, stream>>>(c);
   return cuda_status(cudaGetLastError());
 }
@@ -376,6 +391,8 @@ dsa_status_t launch_indexer_kl(const void* q, const void* kv_cache, const Geomet
   p.num_pages = g.num_pages;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns.load();
+  p.q_start = g.q_start;
+  p.num_q = g.num_q;
   const int64_t grid = (int64_t)g.batch * g.row_count;
   if (grid == 0) return DSA_OK;
   indexer_kl_kernel<<<(unsigned)grid, kKlThreads, kKlSmemBytes, stream>>>(p);
@@ -505,7 +522,7 @@ dsa_status_t launch_selection_mask(const int32_t* idx, int k, const Geometry& g,
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   MaskParams p{idx, g.seqlens, mask, mask_ld, k, g.batch, g.max_ctx, g.q_per_seq, row_begin,
-               row_count};
+               row_count, g.q_start, g.num_q};
   const int64_t grid = (int64_t)g.batch * row_count;
   if (grid == 0) return DSA_OK;
   selection_mask_kernel<<<(unsigned)grid, kMaskThreads, smem, stream>>>(p);
@@ -552,6 +569,8 @@ dsa_status_t launch_masked_mha(const void* q_mha, const void* k_nope, const void
   p.k = k;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns.load();
+  p.q_start = g.q_start;
+  p.num_q = g.num_q;
   const int64_t grid = (int64_t)p.row_blocks * g.batch * kMhaHeads;
   if (grid == 0) return DSA_OK;
   masked_mha_kernel<<<(unsigned)grid, kFaThreads, kFaSmemBytes, stream>>>(p, tm_q, tm_kn, tm_kr,
@@ -573,7 +592,7 @@ dsa_status_t launch_cand_select(const Geometry& g, int row_begin, int row_count,
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   CandParams p{ckey, cpos, cnt, cap, g.seqlens, g.max_ctx, g.q_per_seq, row_begin, row_count,
-               g.batch, k, idx, redo_rows, redo_cnt};
+               g.batch, k, idx, redo_rows, redo_cnt, g.q_start, g.num_q};
   const int64_t grid = (int64_t)g.batch * row_count;
   if (grid == 0) return DSA_OK;
   cand_select_kernel<<<(unsigned)grid, kCandThreads, kCandSmemBytes, stream>>>(p);
@@ -837,7 +856,7 @@ dsa_status_t dsa_indexer_kl(const void* q, const void* kv_cache, const dsa_kv_de
 dsa_status_t dsa_mla_up_project(const void* kv_cache, const void* w_uk, const void* w_uv,
                                 const dsa_kv_desc_t* kv, void* k_nope, void* k_rope, void* v,
                                 int64_t ctx_pad, dsa_stream_t stream) {
-  dsa_q_desc_t qd{kv ? kv->batch : 0, 1, 0, 0};  // keys only: one nominal row per sequence
+  dsa_q_desc_t qd{kv ? kv->batch : 0, 1, 0, 0, nullptr};  // keys only: one nominal row each
   Geometry g;
   dsa_status_t st = check_geometry(kv, &qd, &g);
   if (st != DSA_OK) return st;
@@ -923,7 +942,7 @@ dsa_status_t dsa_mha_prefill(const void* q_idx, const float* w, const void* k_id
   // seqlens array their positions are known here, so the indexer skips them.
   const int r_end = g.row_begin + g.row_count;
   int sel_begin = g.row_begin;
-  if (!g.seqlens)
+  if (!g.seqlens && !g.q_start)
     sel_begin = std::min(r_end, std::max(g.row_begin, k - g.max_ctx + g.q_per_seq));
   const int sel_rows = r_end - sel_begin;
   if (sel_rows > 0) {

@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "rows.cuh"
 
 namespace dsa {
 
@@ -77,23 +78,32 @@ struct IndexerParams {
   int32_t* cand_pos;             // [batch * row_count][cand_cap]
   uint32_t* cand_cnt;            // [batch * row_count], zeroed by the caller
   int32_t cand_cap;
+  const int32_t* q_start;        // [batch + 1] ragged query rows, or nullptr (rows.cuh)
+  int32_t num_q;
   uint64_t timeout_ns;
 };
 
-// One unit: key tiles [kt0, kt1) of the group (sequence b, rows i0 .. i0+nrows-1).
+// One unit: key tiles [kt0, kt1) of the group (sequence b, rows i0 .. i0+nrows-1;
+// the sequence has q_len query rows, the first of them global row t0).
 struct IdxUnit {
-  int b, i0, nrows, seqlen, kt0, kt1;
+  int b, i0, nrows, seqlen, q_len, kt0, kt1;
+  int64_t t0;
 };
 
-// Tiles of group `grp` (0 when its sequence length is invalid) and its geometry.
+// Tiles of group `grp` (0 when its sequence is invalid or has none of the group's
+// rows) and its geometry.
 __device__ __forceinline__ int idx_group(const IndexerParams& p, int grp, IdxUnit& U) {
   U.b = grp / p.groups_per_seq;
   const int g = grp - U.b * p.groups_per_seq;
-  U.seqlen = p.seqlens ? __ldg(p.seqlens + U.b) : p.max_ctx;
-  if (U.seqlen < p.q_per_seq || U.seqlen > p.max_ctx) return 0;
+  const SeqRows R = seq_rows(p.q_start, p.seqlens, U.b, p.q_per_seq, p.num_q, p.max_ctx);
+  if (!R.ok) return 0;
+  U.seqlen = R.seqlen;
+  U.q_len = R.q_len;
+  U.t0 = R.t0;
   U.i0 = p.row_begin + g * p.G;
-  U.nrows = min(p.G, p.row_begin + p.row_count - U.i0);
-  const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
+  U.nrows = min(p.G, min(p.row_begin + p.row_count, R.q_len) - U.i0);
+  if (U.nrows <= 0) return 0;
+  const int pos_max = U.seqlen - U.q_len + U.i0 + U.nrows - 1;
   return (pos_max / kIdxTile) / p.tile_stride + 1;  // tiles 0, S, ..., up to pos_max's
 }
 
@@ -270,7 +280,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     IdxCursor cur{sh.gs, sh.ts};
     IdxUnit U;
     while (!*abort_flag && idx_next(p, sh, cur, U)) {
-      const int pos_max = U.seqlen - p.q_per_seq + U.i0 + U.nrows - 1;
+      const int pos_max = U.seqlen - U.q_len + U.i0 + U.nrows - 1;
       bool ok = true;
       // Paged caches: lane l holds the page of half (l & 1) of tile kb + l / 2
       // for a batch of 16 tiles starting at kb, and the next batch is already
@@ -392,7 +402,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           raw[i] = make_uint4(0u, 0u, 0u, 0u);
           wj[i] = 0.f;
           if (gi < U.nrows) {
-            const int64_t t = (int64_t)U.b * p.q_per_seq + U.i0 + gi;
+            const int64_t t = U.t0 + U.i0 + gi;
             raw[i] = __ldg(reinterpret_cast<const uint4*>(p.q_idx + (t * kIdxHeads + j) * kIdxDim) +
                            hl);
             wj[i] = __ldg(p.w + t * kIdxHeads + j);
@@ -435,11 +445,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const int et = tid - 4 * 32;       // 0..255 among the epilogue threads
     int cpar = 0;                      // filter mode: staging buffer of the next tile
     uint32_t it = 0, un = 0;
-    if (blockIdx.x == 0 && wg == 0) {  // sequences whose length cannot hold their rows
-      for (int b = e; b < p.batch; b += 128) {
-        const int sl = p.seqlens ? __ldg(p.seqlens + b) : p.max_ctx;
-        if (sl < p.q_per_seq || sl > p.max_ctx) report_error(kErrBounds);
-      }
+    if (blockIdx.x == 0 && wg == 0) {  // sequences whose rows or length are out of range
+      for (int b = e; b < p.batch; b += 128)
+        if (!seq_rows(p.q_start, p.seqlens, b, p.q_per_seq, p.num_q, p.max_ctx).ok)
+          report_error(kErrBounds);
     }
     IdxCursor cur{sh.gs, sh.ts};
     IdxUnit U;
@@ -447,7 +456,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       const int qb = un & 1;
       if (!warp_wait(smem_u32(&qfull[qb]), (un >> 1) & 1, TO, abort_flag)) break;
       const float* wrow = wq + qb * 4 * kIdxHeads;
-      const int pos0 = U.seqlen - p.q_per_seq + U.i0;  // position of the group's first row
+      const int pos0 = U.seqlen - U.q_len + U.i0;  // position of the group's first row
       const int pos_max = pos0 + U.nrows - 1;
       float thr_row[4] = {0.f, 0.f, 0.f, 0.f};  // filter mode: the rows' thresholds
       if (kFilter)

@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "rows.cuh"
 
 namespace dsa {
 
@@ -62,6 +63,8 @@ struct KlParams {
   int32_t paged, page_size, max_pages, num_pages;
   float scale_log2;            // scale * log2(e)
   uint64_t timeout_ns;
+  const int32_t* q_start;      // [batch + 1] ragged query rows, or nullptr (rows.cuh)
+  int32_t num_q;
 };
 
 __global__ void __launch_bounds__(kKlThreads, 1) indexer_kl_kernel(const __grid_constant__ KlParams p) {
@@ -89,11 +92,18 @@ __global__ void __launch_bounds__(kKlThreads, 1) indexer_kl_kernel(const __grid_
   const int64_t local = blockIdx.x;                       // row of the window
   const int b = (int)(local / p.row_count);
   const int qi = p.row_begin + (int)(local - (int64_t)b * p.row_count);
-  const int64_t t = (int64_t)b * p.q_per_seq + qi;        // global query row
+  const SeqRows R = seq_rows(p.q_start, p.seqlens, b, p.q_per_seq, p.num_q, p.max_ctx);
+  if (qi >= R.q_len) {  // a window row the sequence does not have (ragged batch): no term
+    if (tid == 0) {
+      if (!R.ok) report_error(kErrBounds);
+      p.kl[local] = 0.f;
+    }
+    return;
+  }
+  const int64_t t = R.t0 + qi;                            // global query row
   const int ntiles = (p.k + kKlTile - 1) / kKlTile;
-  const int seqlen = p.seqlens ? __ldg(p.seqlens + b) : p.max_ctx;
-  const bool seq_ok = seqlen >= p.q_per_seq && seqlen <= p.max_ctx;
-  const int pos = seqlen - p.q_per_seq + qi;
+  const bool seq_ok = R.ok;
+  const int pos = R.seqlen - R.q_len + qi;
 
   if (tid == 0) {
     for (int i = 0; i < kKlStages; ++i) {

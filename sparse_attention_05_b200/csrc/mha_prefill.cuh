@@ -34,6 +34,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "rows.cuh"
 
 namespace dsa {
 
@@ -298,6 +299,8 @@ struct MaskParams {
   uint32_t* mask;          // [T][mask_ld] bits, row t = the global query row
   int64_t mask_ld;         // words per mask row (>= 4 * key tiles)
   int32_t k, batch, max_ctx, q_per_seq, row_begin, row_count;
+  const int32_t* q_start;  // [batch + 1] ragged query rows, or nullptr (rows.cuh)
+  int32_t num_q;
 };
 
 // One CTA per window row. Rows with at most k visible keys select all of them and
@@ -308,10 +311,10 @@ __global__ void __launch_bounds__(kMaskThreads)
   extern __shared__ uint32_t sbits[];
   const int b = (int)(blockIdx.x / p.row_count);
   const int qi = p.row_begin + (int)(blockIdx.x - (int64_t)b * p.row_count);
-  const int64_t t = (int64_t)b * p.q_per_seq + qi;
-  const int seqlen = mha_seqlen(p.seqlens, b, p.max_ctx);
-  if (seqlen < p.q_per_seq || seqlen > p.max_ctx) return;  // the attention reports it
-  const int pos = seqlen - p.q_per_seq + qi;
+  const SeqRows R = seq_rows(p.q_start, p.seqlens, b, p.q_per_seq, p.num_q, p.max_ctx);
+  if (!R.ok || qi >= R.q_len) return;  // the attention reports a bad sequence
+  const int64_t t = R.t0 + qi;
+  const int pos = R.seqlen - R.q_len + qi;
   if (pos + 1 <= p.k) return;
   const int words = ((pos + kMhaTile) / kMhaTile) * 4;  // whole 128-key tiles up to pos
   for (int w = threadIdx.x; w < words; w += kMaskThreads) sbits[w] = 0u;
@@ -347,6 +350,8 @@ struct MhaParams {
   int32_t batch, max_ctx, q_per_seq, row_begin, row_count, row_blocks, k;
   float scale_log2;        // softmax scale * log2(e)
   uint64_t timeout_ns;
+  const int32_t* q_start;  // [batch + 1] ragged query rows, or nullptr (rows.cuh)
+  int32_t num_q;
 };
 
 __global__ void __launch_bounds__(kFaThreads, 1)
@@ -382,11 +387,14 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   const int rb = p.row_blocks - 1 - (int)(blockIdx.x % p.row_blocks);
   const int b = (int)(bh / kMhaHeads), h = (int)(bh % kMhaHeads);
   const int i0 = rb * kMhaTile;  // first window row of the block
-  const int seqlen = mha_seqlen(p.seqlens, b, p.max_ctx);
-  const bool seq_ok = seqlen >= p.q_per_seq && seqlen <= p.max_ctx;
-  const int last_i = min(i0 + kMhaTile, p.row_count) - 1;
-  const int pos_last = seqlen - p.q_per_seq + p.row_begin + last_i;
-  const int nt = (seq_ok && pos_last >= 0) ? pos_last / kMhaTile + 1 : 0;
+  const SeqRows R = seq_rows(p.q_start, p.seqlens, b, p.q_per_seq, p.num_q, p.max_ctx);
+  const bool seq_ok = R.ok;
+  // window rows of this block that the sequence has (a ragged batch's shorter
+  // sequences have fewer than the window)
+  const int rows_here = min(p.row_count, R.q_len - p.row_begin);
+  const int last_i = min(i0 + kMhaTile, rows_here) - 1;
+  const int pos_last = R.seqlen - R.q_len + p.row_begin + last_i;
+  const int nt = (seq_ok && last_i >= i0 && pos_last >= 0) ? pos_last / kMhaTile + 1 : 0;
 
   if (tid == 0) {
     mbar_init(smem_u32(qfull), 1);
@@ -428,7 +436,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_kn);
         prefetch_tmap(&tm_kr);
-        const int t0 = b * p.q_per_seq + p.row_begin + i0;
+        const int t0 = (int)(R.t0 + p.row_begin + i0);
         const uint32_t bar = smem_u32(qfull);
         mbar_arrive_expect_tx(bar, kFaQBytes);
         for (int c = 0; c < 3; ++c) tma_load_3d(smem_u32(sQ + c * kFaQChunk), &tm_q, bar, 64 * c, h, t0);
@@ -519,10 +527,10 @@ __global__ void __launch_bounds__(kFaThreads, 1)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tO = tmem_base + kFaTmemO + lane_off;
     const int i = i0 + r;  // window row
-    const bool row_ok = seq_ok && i < p.row_count;
+    const bool row_ok = seq_ok && i < rows_here;
     const int qi = p.row_begin + i;
-    const int pos = row_ok ? seqlen - p.q_per_seq + qi : -1;  // -1: sees no key
-    const int64_t t = (int64_t)b * p.q_per_seq + qi;
+    const int pos = row_ok ? R.seqlen - R.q_len + qi : -1;  // -1: sees no key
+    const int64_t t = R.t0 + qi;
     const bool use_mask = p.mask != nullptr && row_ok && pos + 1 > p.k;
     const uint4* mrow =
         use_mask ? reinterpret_cast<const uint4*>(p.mask + t * p.mask_ld) : nullptr;

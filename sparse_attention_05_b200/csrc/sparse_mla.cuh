@@ -66,6 +66,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "rows.cuh"
 
 namespace dsa {
 
@@ -140,6 +141,8 @@ struct MlaParams {
   int32_t nseg, seg_keys;
   float* part_o;               // [slots][128][512]
   float* part_lse;             // [slots][128]
+  const int32_t* q_start;      // [batch + 1] ragged query rows, or nullptr (rows.cuh)
+  int32_t num_q;
 };
 
 __global__ void __launch_bounds__(kMlaThreads, 1)
@@ -187,13 +190,18 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   }
   const int b = (int)(local / p.row_count);
   const int qi = p.row_begin + (int)(local - (int64_t)b * p.row_count);
-  const int64_t t = (int64_t)b * p.q_per_seq + qi;  // global query row
+  // Position of this query row and validity of its sequence.
+  const SeqRows R = seq_rows(p.q_start, p.seqlens, b, p.q_per_seq, p.num_q, p.max_ctx);
+  if (qi >= R.q_len) {  // a window row the sequence does not have (ragged batch): both
+    // CTAs of the pair leave before touching any barrier
+    if (!R.ok && tid == 0 && rank == 0) report_error(kErrBounds);
+    return;
+  }
+  const int64_t t = R.t0 + qi;  // global query row
   const int d0 = 256 * (int)rank;        // first value dim (and first key dim) of this CTA
   const int r0 = 512 + 32 * (int)rank;   // this CTA's quarter of the rope dims
-  // Position of this query row and validity of its sequence.
-  const int seqlen = p.seqlens ? __ldg(p.seqlens + b) : p.max_ctx;
-  const bool seq_ok = seqlen >= p.q_per_seq && seqlen <= p.max_ctx;
-  const int pos = seqlen - p.q_per_seq + qi;
+  const bool seq_ok = R.ok;
+  const int pos = R.seqlen - R.q_len + qi;
   // Blocks after the last entry inside [0, pos] hold only masked keys and change
   // nothing (no weight, no new maximum): the cluster stops at that entry's block
   // (the top-k pads a row of fewer than k visible keys with -1 at its end). Only
@@ -744,6 +752,9 @@ struct MlaCombineParams {
   float* lse;
   int64_t n_whole;
   int32_t nseg, row_begin, row_count, q_per_seq;
+  const int32_t* q_start;  // [batch + 1] ragged query rows, or nullptr (rows.cuh)
+  const int32_t* seqlens;
+  int32_t num_q, max_ctx;
 };
 
 // grid (split rows, 16), 256 threads: warp = one of 8 heads, lane = 16 value dims
@@ -754,7 +765,9 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const __grid_constant_
   const int64_t local = p.n_whole + j;
   const int b = (int)(local / p.row_count);
   const int qi = p.row_begin + (int)(local - (int64_t)b * p.row_count);
-  const int64_t t = (int64_t)b * p.q_per_seq + qi;
+  const SeqRows R = seq_rows(p.q_start, p.seqlens, b, p.q_per_seq, p.num_q, p.max_ctx);
+  if (qi >= R.q_len) return;  // no such row: its segments never ran
+  const int64_t t = R.t0 + qi;
   float l[kMlaMaxSeg];
   float m = -INFINITY;
 #pragma unroll

@@ -21,6 +21,7 @@
 #pragma once
 
 #include "ptx.cuh"
+#include "rows.cuh"
 
 namespace dsa {
 
@@ -48,6 +49,8 @@ struct TopkParams {
   // the last tile is -inf where it lies past pos).
   int32_t tile_stride;
   float* kth_out;         // [batch * row_count] or nullptr: the k-th largest score
+  const int32_t* q_start; // [batch + 1] ragged query rows, or nullptr (rows.cuh)
+  int32_t num_q;
 };
 
 // Inverse of score_key (a key back to its fp32 value; +0.0 for a zero).
@@ -202,19 +205,19 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
 
   const int b = blockIdx.x / p.row_count;
   const int i = p.row_begin + blockIdx.x % p.row_count;
-  const int64_t t = (int64_t)b * p.q_per_seq + i;
+  const SeqRows R = seq_rows(p.q_start, p.seqlens, b, p.q_per_seq, p.num_q, p.max_ctx);
+  const int64_t t = R.t0 + i;
   const int tid = threadIdx.x;
-  int32_t* out = p.idx ? p.idx + t * p.k : nullptr;
+  int32_t* out = p.idx && i < R.q_len ? p.idx + t * p.k : nullptr;
 
-  const int seqlen = p.seqlens ? p.seqlens[b] : p.max_ctx;
-  if (seqlen < p.q_per_seq || seqlen > p.max_ctx) {
-    if (tid == 0) report_error(kErrBounds);
+  if (!R.ok || i >= R.q_len) {  // a bad sequence, or a window row it does not have
+    if (!R.ok && tid == 0) report_error(kErrBounds);
     if (out)
       for (int j = tid; j < p.k; j += kTopkThreads) out[j] = -1;
     if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = -INFINITY;
     return;
   }
-  int n = seqlen - p.q_per_seq + i + 1;  // visible keys 0..pos
+  int n = R.seqlen - R.q_len + i + 1;  // visible keys 0..pos
   if (p.tile_stride > 1) n = ((n - 1) / 128 / p.tile_stride + 1) * 128;  // sampled row
   const uint32_t k = (uint32_t)p.k;
   if (n <= p.k) {
@@ -380,9 +383,11 @@ struct CandParams {
   int32_t cand_cap;          // <= kCandCap
   const int32_t* seqlens;    // [batch] or nullptr
   int32_t max_ctx, q_per_seq, row_begin, row_count, batch, k;
-  int32_t* idx;              // [batch * q_per_seq][k]
+  int32_t* idx;              // [num_q][k]
   int32_t* redo_rows;        // [batch * row_count] window rows left to the full path
   uint32_t* redo_cnt;        // how many (zeroed by the caller)
+  const int32_t* q_start;    // [batch + 1] ragged query rows, or nullptr (rows.cuh)
+  int32_t num_q;
 };
 
 constexpr int kCandSmemBytes =
@@ -400,16 +405,17 @@ __global__ void __launch_bounds__(kCandThreads, 2) cand_select_kernel(CandParams
   const int64_t wrow = blockIdx.x;
   const int b = (int)(wrow / p.row_count);
   const int i = p.row_begin + (int)(wrow - (int64_t)b * p.row_count);
-  const int64_t t = (int64_t)b * p.q_per_seq + i;
+  const SeqRows R = seq_rows(p.q_start, p.seqlens, b, p.q_per_seq, p.num_q, p.max_ctx);
+  const int64_t t = R.t0 + i;
   const int tid = threadIdx.x;
-  int32_t* out = p.idx + t * p.k;
-  const int seqlen = p.seqlens ? p.seqlens[b] : p.max_ctx;
-  if (seqlen < p.q_per_seq || seqlen > p.max_ctx) {
-    if (tid == 0) report_error(kErrBounds);
-    for (int j = tid; j < p.k; j += kCandThreads) out[j] = -1;
+  int32_t* out = i < R.q_len ? p.idx + t * p.k : nullptr;
+  if (!R.ok || i >= R.q_len) {  // a bad sequence, or a window row it does not have
+    if (!R.ok && tid == 0) report_error(kErrBounds);
+    if (out)
+      for (int j = tid; j < p.k; j += kCandThreads) out[j] = -1;
     return;
   }
-  const int n = seqlen - p.q_per_seq + i + 1;  // visible keys 0..pos
+  const int n = R.seqlen - R.q_len + i + 1;  // visible keys 0..pos
   if (n <= p.k) {
     for (int j = tid; j < p.k; j += kCandThreads) out[j] = j < n ? j : -1;
     return;

@@ -46,7 +46,8 @@ class KvDescC(ctypes.Structure):
 
 class QDescC(ctypes.Structure):
     _fields_ = [("num_q", ctypes.c_int32), ("q_per_seq", ctypes.c_int32),
-                ("row_begin", ctypes.c_int32), ("row_count", ctypes.c_int32)]
+                ("row_begin", ctypes.c_int32), ("row_count", ctypes.c_int32),
+                ("q_start", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -172,10 +173,16 @@ class KvLayout:
                         num_pages=problem.k_idx.shape[0] if problem.paged else 0)
 
 
-def _qdesc(num_q: int, q_per_seq: int, rows: Optional[Tuple[int, int]] = None) -> QDescC:
-    """rows = (row_begin, row_count) window within each sequence (None = all)."""
+def _qdesc(num_q: int, q_per_seq: int, rows: Optional[Tuple[int, int]] = None,
+           q_start: Optional[torch.Tensor] = None) -> QDescC:
+    """rows = (row_begin, row_count) window within each sequence (None = all);
+    q_start = int32 [batch + 1] device offsets of a ragged batch's query rows
+    (sequence b owns rows q_start[b] .. q_start[b+1] - 1; q_per_seq = the largest
+    count), None for a uniform batch."""
     r0, rc = rows if rows is not None else (0, 0)
-    return QDescC(num_q, q_per_seq, r0, rc)
+    if q_start is not None and (q_start.dtype != torch.int32 or q_start.dim() != 1):
+        raise ValueError("q_start must be a 1-D int32 tensor of batch + 1 offsets")
+    return QDescC(num_q, q_per_seq, r0, rc, _ptr(q_start).value if q_start is not None else None)
 
 
 def round_up(x: int, m: int) -> int:
@@ -196,7 +203,7 @@ def dsa_indexer_scores(q_idx, w, k_idx, k_scale, kv: KvLayout, q_per_seq: int,
     if scores is None:
         scores = torch.empty(kv.batch * _window(kv, q_per_seq, rows), round_up(kv.max_ctx, 128),
                              dtype=torch.float32, device=q_idx.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_indexer_scores(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale),
                                     ctypes.byref(kvd), ctypes.byref(qd), _ptr(scores),
                                     scores.shape[1], _stream(stream)), "dsa_indexer_scores")
@@ -204,12 +211,21 @@ def dsa_indexer_scores(q_idx, w, k_idx, k_scale, kv: KvLayout, q_per_seq: int,
 
 
 def dsa_topk(scores, kv: KvLayout, q_per_seq: int, k: int,
-             idx: Optional[torch.Tensor] = None, rows=None, stream=None) -> torch.Tensor:
-    """Selected positions [T, k] (rows outside the window are left untouched)."""
-    T = kv.batch * q_per_seq
+             idx: Optional[torch.Tensor] = None, rows=None, stream=None, q_start=None,
+             num_q: Optional[int] = None) -> torch.Tensor:
+    """Selected positions [T, k] (rows outside the window are left untouched). A
+    ragged batch (q_start) needs ``idx`` or ``num_q`` for T."""
+    if q_start is None:
+        T = kv.batch * q_per_seq
+    elif num_q is not None:
+        T = num_q
+    elif idx is not None:
+        T = idx.shape[0]
+    else:
+        raise ValueError("dsa_topk on a ragged batch needs idx or num_q")
     if idx is None:
         idx = torch.empty(T, k, dtype=torch.int32, device=scores.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_topk(_ptr(scores), scores.shape[1], ctypes.byref(kvd), ctypes.byref(qd), k,
                           _ptr(idx), _stream(stream)), "dsa_topk")
     return idx
@@ -217,13 +233,13 @@ def dsa_topk(scores, kv: KvLayout, q_per_seq: int, k: int,
 
 def dsa_sparse_mla_fwd(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale: float,
                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                       rows=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                       rows=None, stream=None, q_start=None) -> Tuple[torch.Tensor, torch.Tensor]:
     T = q.shape[0]
     if out is None:
         out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_sparse_mla_fwd(_ptr(q), _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd),
                                     _ptr(idx), idx.shape[1], float(scale), _ptr(out), _ptr(lse),
                                     _stream(stream)), "dsa_sparse_mla_fwd")
@@ -237,7 +253,7 @@ def dsa_sparse_mla_workspace_size() -> int:
 def dsa_sparse_mla_fwd_ws(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale: float,
                           workspace: Optional[torch.Tensor] = None,
                           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                          rows=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                          rows=None, stream=None, q_start=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """dsa_sparse_mla_fwd with scratch for splitting the rows of a partly filled
     last wave (include/dsa.h); ``workspace`` is any 256-B aligned device tensor
     (a fresh one of dsa_sparse_mla_workspace_size() bytes when None)."""
@@ -249,7 +265,7 @@ def dsa_sparse_mla_fwd_ws(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale:
         out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib().dsa_sparse_mla_fwd_ws(_ptr(q), _ptr(kv_cache), ctypes.byref(kvd),
                                        ctypes.byref(qd), _ptr(idx), idx.shape[1], float(scale),
@@ -259,38 +275,39 @@ def dsa_sparse_mla_fwd_ws(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale:
 
 
 def dsa_indexer_kl(q, kv_cache, kv: KvLayout, q_per_seq: int, idx, scale: float, lse, scores,
-                   kl: Optional[torch.Tensor] = None, rows=None, stream=None) -> torch.Tensor:
+                   kl: Optional[torch.Tensor] = None, rows=None, stream=None, q_start=None) -> torch.Tensor:
     """KL(p || softmax(I)) per row of the window (include/dsa.h): idx [T][k], lse
     [T][128] from dsa_sparse_mla_fwd, scores [batch * window rows][ld]."""
     T = q.shape[0]
     if kl is None:
         kl = torch.empty(kv.batch * _window(kv, q_per_seq, rows), dtype=torch.float32,
                          device=q.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_indexer_kl(_ptr(q), _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd),
                                 _ptr(idx), idx.shape[1], float(scale), _ptr(lse), _ptr(scores),
                                 scores.shape[1], _ptr(kl), _stream(stream)), "dsa_indexer_kl")
     return kl
 
 
-def dsa_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None) -> int:
-    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows)
+def dsa_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None,
+                       q_start=None) -> int:
+    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows, q_start)
     return int(lib().dsa_workspace_size(ctypes.byref(kvd), ctypes.byref(qd), k))
 
 
 def dsa_forward(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_per_seq: int, k: int,
                 scale: float, workspace: Optional[torch.Tensor] = None,
                 idx_out: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                lse: Optional[torch.Tensor] = None, rows=None, stream=None):
+                lse: Optional[torch.Tensor] = None, rows=None, stream=None, q_start=None):
     T = q.shape[0]
     if workspace is None:
-        nbytes = dsa_workspace_size(kv, T, q_per_seq, k, rows)
+        nbytes = dsa_workspace_size(kv, T, q_per_seq, k, rows, q_start)
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_forward(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q),
                              _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k, float(scale),
                              _ptr(workspace), workspace.numel(), _ptr(idx_out), _ptr(out),
@@ -301,7 +318,7 @@ def dsa_forward(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_per_seq: 
 def dsa_forward_noalloc(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_per_seq: int,
                         k: int, scale: float, idx_out: Optional[torch.Tensor] = None,
                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                        rows=None, stream=None):
+                        rows=None, stream=None, q_start=None):
     """dsa_forward on the library's own fixed scratch array: the caller passes
     inputs and outputs only (see include/dsa.h for the limits)."""
     T = q.shape[0]
@@ -309,7 +326,7 @@ def dsa_forward_noalloc(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_p
         out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_forward_noalloc(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q),
                                      _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k,
                                      float(scale), _ptr(idx_out), _ptr(out), _ptr(lse),
@@ -320,21 +337,22 @@ def dsa_forward_noalloc(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_p
 # ---- fused indexer -> top-k (no stored score rows) -------------------------------------
 
 
-def dsa_fused_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None) -> int:
-    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows)
+def dsa_fused_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None,
+                             q_start=None) -> int:
+    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows, q_start)
     return int(lib().dsa_fused_workspace_size(ctypes.byref(kvd), ctypes.byref(qd), k))
 
 
 def dsa_select_fused(q_idx, w, k_idx, k_scale, kv: KvLayout, q_per_seq: int, k: int,
-                     cand_cap: int = 0, idx=None, workspace=None, rows=None, stream=None):
+                     cand_cap: int = 0, idx=None, workspace=None, rows=None, stream=None, q_start=None):
     """Selected positions [T, k] without stored score rows (include/dsa.h)."""
     T = q_idx.shape[0]
     if idx is None:
         idx = torch.empty(T, k, dtype=torch.int32, device=q_idx.device)
     if workspace is None:
-        nbytes = dsa_fused_workspace_size(kv, T, q_per_seq, k, rows)
+        nbytes = dsa_fused_workspace_size(kv, T, q_per_seq, k, rows, q_start)
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q_idx.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_select_fused(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale),
                                   ctypes.byref(kvd), ctypes.byref(qd), k, int(cand_cap),
                                   _ptr(workspace), workspace.numel(), _ptr(idx), _stream(stream)),
@@ -344,16 +362,16 @@ def dsa_select_fused(q_idx, w, k_idx, k_scale, kv: KvLayout, q_per_seq: int, k: 
 
 def dsa_forward_fused(q_idx, w, k_idx, k_scale, q, kv_cache, kv: KvLayout, q_per_seq: int,
                       k: int, scale: float, cand_cap: int = 0, workspace=None, idx_out=None,
-                      out=None, lse=None, rows=None, stream=None):
+                      out=None, lse=None, rows=None, stream=None, q_start=None):
     T = q.shape[0]
     if workspace is None:
-        nbytes = dsa_fused_workspace_size(kv, T, q_per_seq, k, rows)
+        nbytes = dsa_fused_workspace_size(kv, T, q_per_seq, k, rows, q_start)
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty(T, HEADS, D_V, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty(T, HEADS, dtype=torch.float32, device=q.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_forward_fused(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q),
                                    _ptr(kv_cache), ctypes.byref(kvd), ctypes.byref(qd), k,
                                    float(scale), int(cand_cap), _ptr(workspace),
@@ -391,12 +409,13 @@ def dsa_mla_up_project(kv_cache, w_uk, w_uv, kv: KvLayout, k_nope=None, k_rope=N
     return k_nope, k_rope, v
 
 
-def dsa_selection_mask(idx, kv: KvLayout, q_per_seq: int, mask=None, rows=None, stream=None):
+def dsa_selection_mask(idx, kv: KvLayout, q_per_seq: int, mask=None, rows=None, stream=None,
+                       q_start=None):
     """Selection bits [T, mask_ld] uint32 (stored as int32) of the window's rows."""
     T, k = idx.shape
     if mask is None:
         mask = torch.zeros(T, mha_ctx_pad(kv) // 32, dtype=torch.int32, device=idx.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_selection_mask(_ptr(idx), k, ctypes.byref(kvd), ctypes.byref(qd),
                                     _ptr(mask), mask.shape[1], _stream(stream)),
            "dsa_selection_mask")
@@ -404,14 +423,14 @@ def dsa_selection_mask(idx, kv: KvLayout, q_per_seq: int, mask=None, rows=None, 
 
 
 def dsa_masked_mha(q_mha, k_nope, k_rope, v, kv: KvLayout, q_per_seq: int, scale: float,
-                   mask=None, k: int = 0, out=None, lse=None, rows=None, stream=None):
+                   mask=None, k: int = 0, out=None, lse=None, rows=None, stream=None, q_start=None):
     """Masked MHA (include/dsa.h): out [T,128,128] bf16, lse [T,128] fp32."""
     T = q_mha.shape[0]
     if out is None:
         out = torch.empty(T, HEADS, MHA_DV, dtype=torch.bfloat16, device=q_mha.device)
     if lse is None:
         lse = torch.empty(T, HEADS, dtype=torch.float32, device=q_mha.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_masked_mha(_ptr(q_mha), _ptr(k_nope), _ptr(k_rope), _ptr(v),
                                 k_nope.shape[2], ctypes.byref(kvd), ctypes.byref(qd), _ptr(mask),
                                 mask.shape[1] if mask is not None else 0, int(k), float(scale),
@@ -419,25 +438,26 @@ def dsa_masked_mha(q_mha, k_nope, k_rope, v, kv: KvLayout, q_per_seq: int, scale
     return out, lse
 
 
-def dsa_mha_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None) -> int:
-    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows)
+def dsa_mha_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None,
+                           q_start=None) -> int:
+    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows, q_start)
     return int(lib().dsa_mha_workspace_size(ctypes.byref(kvd), ctypes.byref(qd), k))
 
 
 def dsa_mha_prefill(q_idx, w, k_idx, k_scale, q_mha, kv_cache, w_uk, w_uv, kv: KvLayout,
                     q_per_seq: int, k: int, scale: float, workspace=None, idx_out=None,
-                    out=None, lse=None, rows=None, stream=None):
+                    out=None, lse=None, rows=None, stream=None, q_start=None):
     """Short-prefill DSA in MHA mode: indexer -> top-k -> masks -> up-projection ->
     masked MHA, one call (include/dsa.h)."""
     T = q_mha.shape[0]
     if workspace is None:
-        nbytes = dsa_mha_workspace_size(kv, T, q_per_seq, k, rows)
+        nbytes = dsa_mha_workspace_size(kv, T, q_per_seq, k, rows, q_start)
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q_mha.device)
     if out is None:
         out = torch.empty(T, HEADS, MHA_DV, dtype=torch.bfloat16, device=q_mha.device)
     if lse is None:
         lse = torch.empty(T, HEADS, dtype=torch.float32, device=q_mha.device)
-    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_mha_prefill(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _ptr(q_mha),
                                  _ptr(kv_cache), _ptr(w_uk), _ptr(w_uv), ctypes.byref(kvd),
                                  ctypes.byref(qd), k, float(scale), _ptr(workspace),

@@ -19,7 +19,8 @@ Shapes (production dims; ``dims`` overrides them):
   seqlens [B]            int32    visible tokens per sequence (incl. the queries)
   block_table [B, max_pages] int32 (paged only)
 Query row t belongs to sequence t // q_per_seq and sits at position
-seqlen - q_per_seq + t % q_per_seq.
+seqlen - q_per_seq + t % q_per_seq; in a ragged batch (``q_start``) sequence b owns
+rows q_start[b] .. q_start[b+1]-1, its last q_start[b+1] - q_start[b] tokens.
 """
 
 from __future__ import annotations
@@ -67,18 +68,31 @@ class Problem:
     block_table: Optional[torch.Tensor] = None
     hot: Optional[torch.Tensor] = None
     name: str = ""
+    # ragged batch: int32 [batch + 1] row offsets (sequence b owns query rows
+    # q_start[b] .. q_start[b+1]-1, its last tokens); q_per_seq is then the largest count
+    q_start: Optional[torch.Tensor] = None
 
     @property
     def num_q(self) -> int:
+        if self.q_start is not None:
+            return int(self.q_start[-1])
         return self.batch * self.q_per_seq
 
+    def q_lens(self) -> torch.Tensor:
+        if self.q_start is not None:
+            qs = self.q_start.cpu().long()
+            return qs[1:] - qs[:-1]
+        return torch.full((self.batch,), self.q_per_seq, dtype=torch.int64)
+
     def q_seq(self) -> torch.Tensor:
-        return torch.arange(self.num_q, dtype=torch.int32) // self.q_per_seq
+        return torch.repeat_interleave(torch.arange(self.batch), self.q_lens()).int()
 
     def q_pos(self) -> torch.Tensor:
-        t = torch.arange(self.num_q)
-        b = t // self.q_per_seq
-        return (self.seqlens.cpu().long()[b] - self.q_per_seq + t % self.q_per_seq).int()
+        lens = self.q_lens()
+        b = torch.repeat_interleave(torch.arange(self.batch), lens)
+        first = torch.cumsum(lens, 0) - lens  # the sequence's first row
+        i = torch.arange(int(lens.sum())) - first[b]
+        return (self.seqlens.cpu().long()[b] - lens[b] + i).int()
 
     def to(self, device) -> "Problem":
         def mv(x):
@@ -86,7 +100,7 @@ class Problem:
         return dataclasses.replace(
             self, q_idx=mv(self.q_idx), w=mv(self.w), k_idx=mv(self.k_idx),
             k_scale=mv(self.k_scale), q=mv(self.q), kv=mv(self.kv), seqlens=mv(self.seqlens),
-            block_table=mv(self.block_table), hot=mv(self.hot))
+            block_table=mv(self.block_table), hot=mv(self.hot), q_start=mv(self.q_start))
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -192,6 +206,45 @@ def paged_decode(batch=128, q_per_seq=2, min_ctx=4096, max_ctx=131072, page_size
                    seqlens=seqlens.to(torch.int32), scale=dims.d_qk ** -0.5, paged=True,
                    page_size=page_size, block_table=block_table,
                    name=f"paged_b{batch}_tq{q_per_seq}_ctx{min_ctx}-{max_ctx}")
+
+
+def ragged(seqlens, q_lens, page_size=64, seed=5, dims=PRODUCTION, device="cpu",
+           latent_std=1.0, w_div=8.0) -> Problem:
+    """A ragged batch on a paged cache: sequence b holds seqlens[b] tokens and its
+    query rows are its last q_lens[b] tokens (q_lens[b] = seqlens[b]: a whole prompt;
+    fewer: a chunk of prefill appended to tokens already cached, or a decode step).
+    Pages are a random permutation of the physical pages; inputs N(0,1) as in the
+    paged decode."""
+    seqlens = torch.as_tensor(seqlens, dtype=torch.int64)
+    q_lens = torch.as_tensor(q_lens, dtype=torch.int64)
+    assert len(seqlens) == len(q_lens) and bool((q_lens <= seqlens).all())
+    g = _gen(seed, device)
+    batch = len(seqlens)
+    max_ctx = int(seqlens.max())
+    pages_per_seq = (seqlens + page_size - 1) // page_size
+    num_pages = int(pages_per_seq.sum())
+    max_pages = (max_ctx + page_size - 1) // page_size
+    perm = torch.randperm(num_pages, generator=g, device=device).to(torch.int32)
+    block_table = torch.full((batch, max_pages), -1, dtype=torch.int32, device=device)
+    off = 0
+    for b, n in enumerate(pages_per_seq.tolist()):
+        block_table[b, :n] = perm[off:off + n]
+        off += n
+    q_start = torch.zeros(batch + 1, dtype=torch.int32)
+    q_start[1:] = torch.cumsum(q_lens, 0).to(torch.int32)
+    T = int(q_start[-1])
+    q_idx = _bf16((T, dims.h_idx, dims.d_idx), g, device)
+    w = _uniform((T, dims.h_idx), g, device) / w_div
+    k_idx, k_scale = _fp8_keys(num_pages * page_size, dims.d_idx, g, device)
+    q = _bf16((T, dims.heads, dims.d_qk), g, device)
+    kv = _bf16((num_pages * page_size, dims.d_qk), g, device, std=latent_std)
+    return Problem(dims=dims, batch=batch, q_per_seq=int(q_lens.max()), max_ctx=max_ctx,
+                   q_idx=q_idx, w=w, k_idx=k_idx.view(num_pages, page_size, dims.d_idx),
+                   k_scale=k_scale.view(num_pages, page_size), q=q,
+                   kv=kv.view(num_pages, page_size, dims.d_qk),
+                   seqlens=seqlens.to(torch.int32).to(device), scale=dims.d_qk ** -0.5,
+                   paged=True, page_size=page_size, block_table=block_table,
+                   q_start=q_start.to(device), name=f"ragged_b{batch}")
 
 
 def tiny(L=256, seed=0, dims=TINY, device="cpu") -> Problem:

@@ -55,8 +55,10 @@ def test_struct_layouts_match_c():
     #include <stddef.h>
     #include "dsa.h"
     int main(void) {
-      printf("%zu %zu %zu %zu %zu\n", sizeof(dsa_kv_desc_t), offsetof(dsa_kv_desc_t, block_table),
-             offsetof(dsa_kv_desc_t, seqlens), sizeof(dsa_q_desc_t), offsetof(dsa_q_desc_t, row_count));
+      printf("%zu %zu %zu %zu %zu %zu\n", sizeof(dsa_kv_desc_t),
+             offsetof(dsa_kv_desc_t, block_table), offsetof(dsa_kv_desc_t, seqlens),
+             sizeof(dsa_q_desc_t), offsetof(dsa_q_desc_t, row_count),
+             offsetof(dsa_q_desc_t, q_start));
       return 0;
     }
     """
@@ -66,7 +68,7 @@ def test_struct_layouts_match_c():
         subprocess.run(["gcc", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
         got = [int(x) for x in subprocess.run([exe], capture_output=True, text=True).stdout.split()]
     want = [ctypes.sizeof(dsa.KvDescC), dsa.KvDescC.block_table.offset, dsa.KvDescC.seqlens.offset,
-            ctypes.sizeof(dsa.QDescC), dsa.QDescC.row_count.offset]
+            ctypes.sizeof(dsa.QDescC), dsa.QDescC.row_count.offset, dsa.QDescC.q_start.offset]
     assert got == want
 
 
@@ -104,6 +106,11 @@ def test_host_argument_checks_without_gpu(lib):
     assert L.dsa_topk(fake, 512, by(kv), by(bad_q), 2048, fake, None) == 1
     # row window outside the sequence
     assert L.dsa_topk(fake, 512, by(kv), by(dsa.QDescC(2, 1, 1, 0)), 2048, fake, None) == 1
+    # ragged batch: more query rows than batch * q_per_seq, or a negative count
+    assert L.dsa_topk(fake, 512, by(kv), by(dsa.QDescC(5, 2, 0, 0, 0x3000)), 2048, fake,
+                      None) == 1
+    assert L.dsa_topk(fake, 512, by(kv), by(dsa.QDescC(-1, 2, 0, 0, 0x3000)), 2048, fake,
+                      None) == 1
     # top-k score rows must be 16-byte aligned
     assert L.dsa_topk(fake, 514, by(kv), by(q), 2048, fake, None) == 1
     # ld below max_ctx rounded to 128
