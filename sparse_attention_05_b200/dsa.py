@@ -197,7 +197,7 @@ def _window(kv: KvLayout, q_per_seq: int, rows) -> int:
 
 def dsa_indexer_scores(q_idx, w, k_idx, k_scale, kv: KvLayout, q_per_seq: int,
                        scores: Optional[torch.Tensor] = None, rows=None,
-                       stream=None) -> torch.Tensor:
+                       stream=None, q_start=None) -> torch.Tensor:
     """Scores [batch * window_rows, ld] (window rows stored compactly)."""
     T = q_idx.shape[0]
     if scores is None:

@@ -172,3 +172,16 @@ def test_workspace_size_includes_the_split_rows(lib, batch, q_per_seq, max_ctx, 
     part = -(-n_split * nseg * MLA_PART_BYTES // 256) * 256
     assert n == idx + max(score, part)
     assert lib.dsa_sparse_mla_workspace_size() == 74 * MLA_PART_BYTES
+
+
+def test_every_binding_call_that_forwards_q_start_accepts_it():
+    """Each wrapper that builds a query descriptor takes the ragged offsets."""
+    import inspect
+    from sparse_attention_05_b200 import dsa
+    for name in sorted(dsa.SIGNATURES):
+        fn = getattr(dsa, name, None)
+        if fn is None:
+            continue
+        src = inspect.getsource(fn)
+        if "_qdesc(" in src:
+            assert "q_start" in inspect.signature(fn).parameters, name
