@@ -326,7 +326,8 @@ class Runner:
     """Holds the device buffers of one workload and runs one step of the path
     through the library's stage calls (the same launches dsa_forward makes)."""
 
-    def __init__(self, p: synth.Problem, k: int = K_SEL, with_kl: bool = False):
+    def __init__(self, p: synth.Problem, k: int = K_SEL, with_kl: bool = False,
+                 split_topk: bool = False):
         from sparse_attention_05_b200 import dsa
         self.dsa = dsa
         self.p = p
@@ -350,6 +351,12 @@ class Runner:
         self.out = torch.empty(T, 128, 512, dtype=torch.bfloat16, device=p.q.device)
         self.lse = torch.empty(T, 128, dtype=torch.float32, device=p.q.device)
         self.mla_ws = self.ws
+        # the selection dsa_forward makes: one CTA per row (dsa_topk); with --split-topk
+        # the split path of dsa_topk_ws (threshold, chunk sweep, per-row selection)
+        tk = (dsa.dsa_topk_workspace_size(self.kv, T, p.q_per_seq, k, rows=(0, rows))
+              if split_topk else 0)
+        self.topk_ws = torch.empty(max(tk, 256), dtype=torch.uint8, device=p.q.device)
+        self.topk_launches = 3 if tk else 1
         self.with_kl = with_kl
         if with_kl:
             if len(self.chunks) > 1:
@@ -358,8 +365,9 @@ class Runner:
             # the KL term reads the score rows after the attention: keep them intact
             self.mla_ws = torch.empty(dsa.dsa_sparse_mla_workspace_size(), dtype=torch.uint8,
                                       device=p.q.device)
-        self.launches_per_step = (2 * len(self.chunks) + mla_split_launches(T, k, self.mla_ws.numel())
-                                  + (1 if with_kl else 0))
+        self.launches_per_step = ((1 + self.topk_launches) * len(self.chunks) +
+                                  mla_split_launches(T, k, self.mla_ws.numel()) +
+                                  (1 if with_kl else 0))
 
     def step(self, ev=None):
         d, p = self.dsa, self.p
@@ -371,8 +379,7 @@ class Runner:
             if ev is not None:
                 ev["indexer"].append(_record())
                 ev["topk"].append(_record())
-            d.dsa_topk(self.scores[: p.batch * rc], self.kv, p.q_per_seq, self.k, idx=self.idx,
-                       rows=(r0, rc))
+            self.topk(r0, rc)
             if ev is not None:
                 ev["topk"].append(_record())
         if ev is not None:
@@ -388,6 +395,15 @@ class Runner:
                              self.scores, kl=self.kl)
             if ev is not None:
                 ev["indexer_kl"].append(_record())
+
+    def topk(self, r0, rc):
+        d, p = self.dsa, self.p
+        if self.topk_launches > 1:
+            d.dsa_topk_ws(self.scores[: p.batch * rc], self.kv, p.q_per_seq, self.k,
+                          workspace=self.topk_ws, idx=self.idx, rows=(r0, rc))
+        else:
+            d.dsa_topk(self.scores[: p.batch * rc], self.kv, p.q_per_seq, self.k, idx=self.idx,
+                       rows=(r0, rc))
 
     # end-to-end through the public call dsa_forward
     def e2e_host_inputs(self):
@@ -427,7 +443,7 @@ class CpRunner(Runner):
             per &= ~3
         self.chunks = [(r0 + c, min(per, rc - c)) for r0, rc in self.windows
                        for c in range(0, rc, per)]
-        self.launches_per_step = 2 * len(self.chunks) + len(self.windows)
+        self.launches_per_step = (1 + self.topk_launches) * len(self.chunks) + len(self.windows)
 
     def step(self, ev=None):
         d, p = self.dsa, self.p
@@ -446,8 +462,7 @@ class CpRunner(Runner):
             if ev is not None:
                 ev["indexer"].append(_record())
                 ev["topk"].append(_record())
-            d.dsa_topk(self.scores[: p.batch * rc], self.kv, p.q_per_seq, self.k, idx=self.idx,
-                       rows=(r0, rc))
+            self.topk(r0, rc)
             if ev is not None:
                 ev["topk"].append(_record())
         for r0, rc in self.windows:
@@ -940,6 +955,9 @@ def main(argv=None):
                     help="fused indexer -> top-k selection (no stored score rows)")
     ap.add_argument("--mode", default="mqa", choices=["mqa", "mha"],
                     help="mha: short-prefill DSA in MLA's MHA mode (masked MHA; prefill_8k)")
+    ap.add_argument("--split-topk", action="store_true",
+                    help="time the split selection of dsa_topk_ws (long rows swept by several "
+                         "CTAs) instead of dsa_forward's one CTA per row")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the 128K prefill half of the metric in the default run")
     ap.add_argument("--no-fp8-peak", action="store_true",
@@ -983,7 +1001,7 @@ def main(argv=None):
         r = MhaRunner(p, seed=rank)
         work = algorithmic_work_mha(p)
     else:
-        r = Runner(p, with_kl=args.kl)
+        r = Runner(p, with_kl=args.kl, split_topk=args.split_topk)
         work = algorithmic_work(p)
     peaks = load_peaks()
 

@@ -142,6 +142,21 @@ DSA_API dsa_status_t dsa_indexer_scores(const void* q_idx, const float* w, const
 DSA_API dsa_status_t dsa_topk(const float* scores, int64_t ld, const dsa_kv_desc_t* kv,
                       const dsa_q_desc_t* q, int32_t k, int32_t* idx, dsa_stream_t stream);
 
+/* dsa_topk with a scratch buffer that lets long rows be swept by several CTAs at
+ * once (the same selection, bit for bit). Rows of more than 4k visible keys are cut
+ * into chunks of 16384 keys; each chunk's CTA keeps the keys at or above the row's
+ * sample threshold (the one dsa_topk uses) as candidates, and one CTA per row then
+ * selects the exact top k from the candidates, or from the whole row when the
+ * candidates cannot decide it. Applies when max_ctx <= 131072; otherwise, or with a
+ * workspace smaller than dsa_topk_workspace_size(), the call is dsa_topk.
+ *  workspace  device, 256-byte aligned, or NULL; the library writes it during the
+ *             call (stream order) and keeps nothing in it afterwards.
+ * Other arguments as dsa_topk. */
+DSA_API size_t dsa_topk_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k);
+DSA_API dsa_status_t dsa_topk_ws(const float* scores, int64_t ld, const dsa_kv_desc_t* kv,
+                                 const dsa_q_desc_t* q, int32_t k, void* workspace,
+                                 size_t workspace_bytes, int32_t* idx, dsa_stream_t stream);
+
 /* Sparse MLA forward in MQA mode (report §1 Eq. 2, Fig. 1).
  *  q     bf16 [T][128][576] absorbed queries
  *  kv    bf16 latent cache, [B][max_ctx][576] or paged [num_pages][page_size][576]
@@ -208,7 +223,8 @@ DSA_API size_t dsa_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q
  * dsa_workspace_size() bytes let the score rows go in chunks of up to 2 GiB. A
  * smaller workspace is accepted down to the indices plus one score row per
  * sequence; the rows are then processed in smaller chunks. Too small a
- * workspace returns DSA_ERR_WORKSPACE. Once the selection is done, the space of the
+ * workspace returns DSA_ERR_WORKSPACE. The selection is dsa_topk's (one CTA per
+ * row). Once the selection is done, the space of the
  * score rows serves the sparse MLA as dsa_sparse_mla_fwd_ws's scratch (split rows of
  * a partly filled last wave); dsa_workspace_size() includes what that needs.
  * idx_out (int32 [T][k]) receives the selection when not NULL. */

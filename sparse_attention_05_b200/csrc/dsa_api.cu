@@ -32,6 +32,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 dsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
 // Validated geometry shared by every entry point.
 struct Geometry {
   int layout, batch, max_ctx, page_size, num_pages, max_pages, q_per_seq, num_q;
@@ -143,6 +145,76 @@ dsa_status_t launch_topk(const float* scores, int64_t ld, const Geometry& g, int
   const int64_t grid = (int64_t)g.batch * row_count;
   if (grid == 0) return DSA_OK;
   topk_kernel<<<(unsigned)grid, kTopkThreads, kTopkSmemBytes, stream>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+// ---- split top-k (long rows swept by several CTAs) ----------------------------------
+// Scratch of the split path for `rows` window rows: each row's candidate keys and
+// positions (kCandCap each), then the rows' candidate counts and threshold keys.
+size_t split_topk_bytes(int64_t rows) {
+  return align256((size_t)rows * kCandCap * 8) + 2 * align256((size_t)rows * 4);
+}
+
+// Whether the split path applies: some row may hold more than 4k keys (else the
+// one-CTA kernel has nothing to split), every row fits the selection bitmaps, and
+// the rows are few enough that one CTA per row would leave SMs idle (with many rows,
+// as in prefill, every SM is busy anyway and splitting only adds launches).
+// dsa_forward's choice between the two selections. Measured on B200 (paged 128K
+// decode, 256 rows): the split path's threshold, sweep and select kernels take 16 +
+// 36 + 28 us against 78 us for one CTA per row (each of the three is bound by fixed
+// latency: short-lived sweep CTAs in waves, and the block-wide radix passes of the
+// threshold and of the selection), so the forward keeps one CTA per row; the split
+// path stays available through dsa_topk_ws.
+constexpr bool kForwardSplitTopk = false;
+
+bool split_topk_applies(const Geometry& g, int k) {
+  return g.max_ctx > 4 * k && g.max_ctx <= kCandMaxWords * 32 &&
+         (int64_t)g.batch * g.row_count <= 4 * (int64_t)num_sms();
+}
+
+dsa_status_t launch_topk_split(const float* scores, int64_t ld, const Geometry& g,
+                               int row_begin, int row_count, int k, int32_t* idx,
+                               cudaStream_t stream, void* scratch) {
+  static DeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [] {
+    cudaError_t e = cudaFuncSetAttribute(topk_threshold_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kThresholdSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSelectSmemBytes);
+    return e;
+  });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  const int64_t rows = (int64_t)g.batch * row_count;
+  if (rows == 0) return DSA_OK;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(scratch);
+  SplitParams p{};
+  p.scores = scores;
+  p.ld = ld;
+  p.seqlens = g.seqlens;
+  p.q_start = g.q_start;
+  p.num_q = g.num_q;
+  p.max_ctx = g.max_ctx;
+  p.q_per_seq = g.q_per_seq;
+  p.row_begin = row_begin;
+  p.row_count = row_count;
+  p.batch = g.batch;
+  p.k = k;
+  p.nchunk = (g.max_ctx + kSplitChunk - 1) / kSplitChunk;
+  p.cand_key = reinterpret_cast<uint32_t*>(ws);
+  p.cand_pos = reinterpret_cast<int32_t*>(ws + (size_t)rows * kCandCap * 4);
+  p.cand_cnt = reinterpret_cast<uint32_t*>(ws + align256((size_t)rows * kCandCap * 8));
+  p.thr_key = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.cand_cnt) +
+                                          align256((size_t)rows * 4));
+  p.idx = idx;
+  topk_threshold_kernel<<<(unsigned)rows, kTopkThreads, kThresholdSmemBytes, stream>>>(p);
+  dsa_status_t st = cuda_status(cudaGetLastError());
+  if (st != DSA_OK) return st;
+  topk_sweep_kernel<<<(unsigned)(rows * p.nchunk), kTopkThreads, 0, stream>>>(p);
+  st = cuda_status(cudaGetLastError());
+  if (st != DSA_OK) return st;
+  topk_select_kernel<<<(unsigned)rows, kTopkThreads, kSelectSmemBytes, stream>>>(p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -409,7 +481,6 @@ struct ForwardPlan {
   size_t score_bytes;   // one chunk of score rows
 };
 
-inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 ForwardPlan plan_forward(const Geometry& g, int k, bool need_idx) {
   ForwardPlan f;
@@ -764,10 +835,13 @@ size_t dsa_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_
   Geometry g;
   if (check_geometry(kv, q, &g) != DSA_OK || k < 1 || k > kMaxK) return 0;
   const ForwardPlan f = plan_forward(g, k, true);
+  // the split top-k's candidates follow a chunk's score rows
+  const size_t split = kForwardSplitTopk && split_topk_applies(g, k)
+                           ? split_topk_bytes((int64_t)f.chunk_rows * g.batch) : 0;
   // after the selection the score space holds the sparse MLA's split rows
   const MlaSplit sp = plan_mla_split((int64_t)g.batch * g.row_count, k, SIZE_MAX);
   const size_t part_bytes = (size_t)(sp.n_split * sp.nseg) * kMlaPartBytes;
-  return f.idx_bytes + std::max(f.score_bytes, align256(part_bytes));
+  return f.idx_bytes + std::max(f.score_bytes + split, align256(part_bytes));
 }
 
 dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
@@ -789,11 +863,26 @@ dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
       workspace_bytes < f.idx_bytes)
     return DSA_ERR_WORKSPACE;
-  // A smaller workspace than dsa_workspace_size() is accepted: the score rows
-  // are then processed in smaller chunks (down to one row per sequence).
-  if (workspace_bytes < f.idx_bytes + f.score_bytes) {
-    const int64_t row_bytes = f.ld * 4 * g.batch;
-    int64_t rows = (int64_t)(workspace_bytes - f.idx_bytes) / row_bytes;
+  // Long rows take the split top-k when its candidate scratch fits after the score
+  // rows. A smaller workspace than dsa_workspace_size() is accepted: the score rows
+  // are then processed in smaller chunks (down to one row per sequence), with the
+  // split top-k while its scratch still fits beside them, else without it.
+  const int64_t row_bytes = f.ld * 4 * g.batch;
+  const size_t avail = workspace_bytes - f.idx_bytes;
+  bool split = kForwardSplitTopk && split_topk_applies(g, k);
+  if (split && avail < f.score_bytes + split_topk_bytes((int64_t)f.chunk_rows * g.batch)) {
+    const int64_t per_row = row_bytes + (int64_t)g.batch * (kCandCap * 8 + 4);
+    int64_t rows = std::min<int64_t>(f.chunk_rows, ((int64_t)avail - 1024) / per_row);
+    if (rows >= 4) rows &= ~int64_t(3);
+    if (rows >= 1) {
+      f.chunk_rows = (int)rows;
+      f.score_bytes = align256((size_t)rows * row_bytes);
+    } else {
+      split = false;
+    }
+  }
+  if (!split && avail < f.score_bytes) {
+    int64_t rows = (int64_t)avail / row_bytes;
     if (rows < 1) return DSA_ERR_WORKSPACE;
     if (rows >= 4) rows &= ~int64_t(3);
     f.chunk_rows = (int)rows;
@@ -801,13 +890,15 @@ dsa_status_t dsa_forward(const void* q_idx, const float* w, const void* k_idx,
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws);
   float* scores = reinterpret_cast<float*>(ws + f.idx_bytes);
+  void* split_ws = ws + f.idx_bytes + f.score_bytes;
   cudaStream_t s = (cudaStream_t)stream;
   const int r_end = g.row_begin + g.row_count;
   for (int r0 = g.row_begin; r0 < r_end; r0 += f.chunk_rows) {
     const int rc = std::min(f.chunk_rows, r_end - r0);
     st = launch_indexer(q_idx, w, k_idx, k_scale, g, scores, f.ld, r0, rc, s);
     if (st != DSA_OK) return st;
-    st = launch_topk(scores, f.ld, g, r0, rc, k, idx, s);
+    st = split ? launch_topk_split(scores, f.ld, g, r0, rc, k, idx, s, split_ws)
+               : launch_topk(scores, f.ld, g, r0, rc, k, idx, s);
     if (st != DSA_OK) return st;
   }
   // the score rows are dead once the last top-k has run (stream order): their
@@ -1113,6 +1204,29 @@ dsa_status_t dsa_get_device_error(dsa_stream_t stream) {
     if (e != cudaSuccess) return DSA_ERR_CUDA;
   }
   return (dsa_status_t)word;
+}
+
+size_t dsa_topk_workspace_size(const dsa_kv_desc_t* kv, const dsa_q_desc_t* q, int32_t k) {
+  Geometry g;
+  if (check_geometry(kv, q, &g) != DSA_OK || k < 1 || k > kMaxK) return 0;
+  return split_topk_applies(g, k) ? split_topk_bytes((int64_t)g.batch * g.row_count) : 0;
+}
+
+dsa_status_t dsa_topk_ws(const float* scores, int64_t ld, const dsa_kv_desc_t* kv,
+                         const dsa_q_desc_t* q, int32_t k, void* workspace,
+                         size_t workspace_bytes, int32_t* idx, dsa_stream_t stream) {
+  Geometry g;
+  dsa_status_t st = check_geometry(kv, q, &g);
+  if (st != DSA_OK) return st;
+  if (!scores || !idx) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (ld < g.max_ctx || ld % 4 != 0 || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+  const int64_t rows = (int64_t)g.batch * g.row_count;
+  if (workspace && split_topk_applies(g, k) && workspace_bytes >= split_topk_bytes(rows))
+    return launch_topk_split(scores, ld, g, g.row_begin, g.row_count, k, idx,
+                             (cudaStream_t)stream, workspace);
+  return launch_topk(scores, ld, g, g.row_begin, g.row_count, k, idx, (cudaStream_t)stream);
 }
 
 dsa_status_t dsa_topk(const float* scores, int64_t ld, const dsa_kv_desc_t* kv,

@@ -194,6 +194,45 @@ __device__ void compact_topk(int n, uint32_t tau, uint32_t r_eq, KeyAt key_at, P
   }
 }
 
+// A row of k < n <= 4k <= 8192 keys: staged in shared memory `cache` (all loads in
+// flight; rows start 16-B aligned), then the exact top k selected from it. The k-th
+// score goes to *kth when kth is given; the selection to out when out is given.
+__device__ void select_short_row(const float* row, int n, uint32_t k, float* cache,
+                                 uint32_t* hist, uint32_t* misc, int32_t* out, float* kth) {
+  const int tid = threadIdx.x;
+  {
+    constexpr int kPer = 4 * kTopkThreads;
+    constexpr int kLoads = 8192 / kPer;  // n <= 4k <= 8192
+    float4 v[kLoads];
+#pragma unroll
+    for (int h = 0; h < kLoads; ++h) {
+      const int e0 = h * kPer + 4 * tid;
+      if (e0 + 3 < n) {
+        v[h] = *reinterpret_cast<const float4*>(row + e0);
+      } else {
+        v[h].x = e0 < n ? row[e0] : -INFINITY;
+        v[h].y = e0 + 1 < n ? row[e0 + 1] : -INFINITY;
+        v[h].z = e0 + 2 < n ? row[e0 + 2] : -INFINITY;
+        v[h].w = e0 + 3 < n ? row[e0 + 3] : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kLoads; ++h) {
+      const int e0 = h * kPer + 4 * tid;
+      if (e0 < n) *reinterpret_cast<float4*>(cache + e0) = v[h];
+    }
+    for (int e0 = kLoads * kPer + 4 * tid; e0 < n; e0 += kPer)  // not reached for k <= 2048
+      for (int u = 0; u < 4 && e0 + u < n; ++u) cache[e0 + u] = row[e0 + u];
+    __syncthreads();
+  }
+  uint32_t tau, r_eq;
+  find_kth(n, k, [&](int e, int) { return score_key(cache[e]); }, hist, misc, tau, r_eq);
+  if (kth && tid == 0) *kth = key_score(tau);
+  if (out)
+    compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(cache[e]); },
+                 [&](int e) { return e; }, out, misc);
+}
+
 __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* cache = reinterpret_cast<float*>(smem_raw);
@@ -327,38 +366,8 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
     return;
   }
 
-  // ---- short rows: staged in shared memory (all loads in flight), then selected ----
-  // (n <= 4k <= 8192 <= kTopkCacheElems; rows start 16-B aligned)
-  {
-    constexpr int kPer = 4 * kTopkThreads;
-    constexpr int kLoads = 8192 / kPer;  // n <= 4k <= 8192
-    float4 v[kLoads];
-#pragma unroll
-    for (int h = 0; h < kLoads; ++h) {
-      const int e0 = h * kPer + 4 * tid;
-      if (e0 + 3 < n) {
-        v[h] = *reinterpret_cast<const float4*>(row + e0);
-      } else {
-        v[h].x = e0 < n ? row[e0] : -INFINITY;
-        v[h].y = e0 + 1 < n ? row[e0 + 1] : -INFINITY;
-        v[h].z = e0 + 2 < n ? row[e0 + 2] : -INFINITY;
-        v[h].w = e0 + 3 < n ? row[e0 + 3] : -INFINITY;
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < kLoads; ++h) {
-      const int e0 = h * kPer + 4 * tid;
-      if (e0 < n) *reinterpret_cast<float4*>(cache + e0) = v[h];
-    }
-    for (int e0 = kLoads * kPer + 4 * tid; e0 < n; e0 += kPer)  // not reached for k <= 2048
-      for (int u = 0; u < 4 && e0 + u < n; ++u) cache[e0 + u] = row[e0 + u];
-    __syncthreads();
-  }
-  find_kth(n, k, [&](int e, int) { return score_key(cache[e]); }, hist, misc, tau, r_eq);
-  if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = key_score(tau);
-  if (out)
-    compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(cache[e]); },
-                 [&](int e) { return e; }, out, misc);
+  // ---- short rows: staged in shared memory, then selected ----
+  select_short_row(row, n, k, cache, hist, misc, out, p.kth_out ? p.kth_out + blockIdx.x : nullptr);
 }
 
 // ======================================================================================
@@ -373,6 +382,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
 // the keys equal to tau marked from a second bitmap, and the marks compacted in
 // ascending order. Other rows are listed for the full (unfused) selection.
 constexpr int kCandThreads = 512;
+static_assert(kCandThreads == kTopkThreads, "the shared selection code assumes one block shape");
 constexpr int kCandCap = 8192;                     // candidates per row staged in smem
 constexpr int kCandMaxWords = 4096;                // bitmap words: rows of <= 131072 keys
 
@@ -392,6 +402,61 @@ struct CandParams {
 
 constexpr int kCandSmemBytes =
     kCandCap * 8 + 2 * kCandMaxWords * 4 + 2048 * 4 + 64 * 4;
+
+// The exact top k of a row of n visible keys from m >= k candidates staged in
+// shared memory as (order-preserving key, position) in any order, when they hold
+// every key of the row at or above the row's k-th key: the k-th key tau and the
+// number r of equal keys to take (find_kth), keys above tau marked in a bitmap over
+// the row's positions, the r lowest positions among the keys equal to tau marked
+// from a second bitmap, and the marks compacted in ascending order into out.
+// Bitmaps of (n + 31) / 32 <= kCandMaxWords words.
+__device__ void select_from_candidates(int m, int n, uint32_t k, const uint32_t* ckey,
+                                       const int32_t* cpos, uint32_t* sel, uint32_t* tie,
+                                       uint32_t* hist, uint32_t* misc, int32_t* out) {
+  const int tid = threadIdx.x;
+  const int words = (n + 31) >> 5;
+  for (int w = tid; w < words; w += kTopkThreads) sel[w] = tie[w] = 0u;
+  __syncthreads();
+  uint32_t tau, r_eq;
+  find_kth(m, k, [&](int e, int) { return ckey[e]; }, hist, misc, tau, r_eq);
+  for (int e = tid; e < m; e += kTopkThreads) {
+    const uint32_t key = ckey[e];
+    const int pos = cpos[e];
+    if (key > tau) atomicOr(&sel[pos >> 5], 1u << (pos & 31));
+    else if (key == tau) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+  }
+  __syncthreads();
+  // the r_eq lowest positions among the keys equal to tau: an ordered scan of the
+  // tie bitmap (each thread owns consecutive words)
+  const int per = (words + kTopkThreads - 1) / kTopkThreads;
+  const int w0 = tid * per;
+  uint32_t cnt = 0;
+  for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(tie[w]);
+  uint32_t before = block_exclusive_scan(cnt, misc, misc + 32);
+  for (int w = w0; w < w0 + per && w < words; ++w) {
+    uint32_t bits = tie[w];
+    while (bits) {
+      const uint32_t bit = bits & (~bits + 1u);
+      if (before < r_eq) sel[w] |= bit;
+      ++before;
+      bits ^= bit;
+    }
+  }
+  __syncthreads();
+  // ascending compaction of the selection (exactly k marks)
+  cnt = 0;
+  for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(sel[w]);
+  uint32_t o = block_exclusive_scan(cnt, misc, misc + 32);
+  for (int w = w0; w < w0 + per && w < words; ++w) {
+    uint32_t bits = sel[w];
+    while (bits) {
+      const int bpos = __ffs(bits) - 1;
+      if (o < k) out[o] = w * 32 + bpos;
+      ++o;
+      bits &= bits - 1u;
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kCandThreads, 2) cand_select_kernel(CandParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -428,52 +493,227 @@ __global__ void __launch_bounds__(kCandThreads, 2) cand_select_kernel(CandParams
     }
     return;
   }
-  const int words = (n + 31) >> 5;  // <= kCandMaxWords (checked on the host)
   for (uint32_t e = tid; e < m; e += kCandThreads) {
     ckey[e] = p.cand_key[wrow * p.cand_cap + e];
     cpos[e] = p.cand_pos[wrow * p.cand_cap + e];
   }
-  for (int w = tid; w < words; w += kCandThreads) sel[w] = tie[w] = 0u;
+  select_from_candidates((int)m, n, (uint32_t)p.k, ckey, cpos, sel, tie, hist, misc, out);
+}
+
+
+// ======================================================================================
+// Long rows split across CTAs (the unfused selection with a scratch buffer)
+// ======================================================================================
+// One CTA per row holds a long row's whole sweep: a 131072-key row takes 16 sweep
+// steps of 8192 keys one after the other, and with few rows (decode) the longest
+// rows alone set the time. Here the sweep of a row with more than 4k keys is cut
+// into chunks of kSplitChunk keys, one CTA each (topk_sweep_kernel): each chunk CTA
+// takes the row threshold (computed once per row by topk_threshold_kernel from the
+// same strided sample of 2048 scores as the one-CTA path) and appends the keys of its
+// chunk at or above it to the row's candidate list with one atomic per warp and step
+// (no block barrier per step, in no particular order). topk_select_kernel then selects per row: rows of at most 4k
+// keys from their scores staged in shared memory, long rows from their candidates
+// (select_from_candidates) when there are at least k of them and no more than the
+// list holds -- they then hold every key at or above the row's k-th -- and the
+// others by the exact full-row path. The result equals topk_kernel's bit for bit.
+constexpr int kSplitChunk = 16384;  // keys per sweep CTA (64 KB of scores)
+
+struct SplitParams {
+  const float* scores;     // [batch * row_count][ld]
+  int64_t ld;
+  const int32_t* seqlens;  // [batch] or nullptr
+  const int32_t* q_start;  // [batch + 1] ragged query rows, or nullptr (rows.cuh)
+  int32_t num_q, max_ctx, q_per_seq, row_begin, row_count, batch, k;
+  int32_t nchunk;          // sweep chunks per window row: ceil(max_ctx / kSplitChunk)
+  uint32_t* cand_key;      // [batch * row_count][kCandCap]
+  int32_t* cand_pos;       // [batch * row_count][kCandCap]
+  uint32_t* cand_cnt;      // [batch * row_count], zeroed by topk_threshold_kernel
+  uint32_t* thr_key;       // [batch * row_count] long rows' threshold keys
+  int32_t* idx;            // [num_q][k] (topk_select_kernel)
+};
+
+// Window row `wrow` of the split top-k: its global row t and visible keys n (0 when
+// the row does not exist or its sequence is invalid).
+__device__ __forceinline__ int split_row(const SplitParams& p, int64_t wrow, int64_t& t,
+                                         bool& ok) {
+  const int b = (int)(wrow / p.row_count);
+  const int i = p.row_begin + (int)(wrow - (int64_t)b * p.row_count);
+  const SeqRows R = seq_rows(p.q_start, p.seqlens, b, p.q_per_seq, p.num_q, p.max_ctx);
+  t = R.t0 + i;
+  ok = R.ok;
+  if (!R.ok || i >= R.q_len) return 0;
+  return R.seqlen - R.q_len + i + 1;
+}
+
+// Threshold key of a long row: the r-th largest of the fixed strided sample of 2048
+// scores, r = expected count of top-k keys in the sample + 4 standard deviations + 16
+// (the same threshold the one-CTA path of topk_kernel uses).
+__device__ __forceinline__ uint32_t long_row_threshold(const float* row, int n, uint32_t k,
+                                                       uint32_t* sample, uint32_t* hist,
+                                                       uint32_t* misc) {
+  for (int s = threadIdx.x; s < kTopkSample; s += kTopkThreads)
+    sample[s] = score_key(row[(int64_t)s * n / kTopkSample]);
   __syncthreads();
+  const float expect = (float)k / (float)n * kTopkSample;
+  uint32_t r = (uint32_t)(expect + 4.0f * sqrtf(expect) + 16.0f);
+  r = min(r, (uint32_t)kTopkSample);
+  uint32_t tau_low, unused;
+  find_kth(kTopkSample, r, [&](int e, int) { return sample[e]; }, hist, misc, tau_low, unused);
+  return tau_low;
+}
+
+constexpr int kThresholdSmemBytes = 2048 * 4 + 64 * 4 + kTopkSample * 4;
+
+// One CTA per window row: zeroes the row's candidate count and, for a long row,
+// computes its threshold key once for all of its chunk CTAs.
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_threshold_kernel(SplitParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
+  uint32_t* misc = hist + 2048;
+  uint32_t* sample = misc + 64;
+  const int64_t wrow = blockIdx.x;
+  int64_t t;
+  bool ok;
+  const int n = split_row(p, wrow, t, ok);
+  if (threadIdx.x == 0) p.cand_cnt[wrow] = 0u;
+  if (n <= 4 * p.k) return;
+  const uint32_t thr =
+      long_row_threshold(p.scores + wrow * p.ld, n, (uint32_t)p.k, sample, hist, misc);
+  if (threadIdx.x == 0) p.thr_key[wrow] = thr;
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_sweep_kernel(SplitParams p) {
+  const int64_t wrow = blockIdx.x / p.nchunk;
+  const int chunk = (int)(blockIdx.x - wrow * p.nchunk);
+  int64_t t;
+  bool ok;
+  const int n = split_row(p, wrow, t, ok);
+  const int c0 = chunk * kSplitChunk;
+  if (n <= 4 * p.k || c0 >= n) return;  // short rows and chunks past the row: no sweep
+  const int c1 = min(n, c0 + kSplitChunk);
+  const float* row = p.scores + wrow * p.ld;
+  const float thr = key_score(p.thr_key[wrow]);
+  // 16 consecutive keys per thread per step (8192 keys), both steps' loads issued
+  // before either is used; keys >= thr <=> key >= threshold key (no NaN scores)
+  const int tid = threadIdx.x, lane = tid & 31;
+  constexpr int kStep = 16 * kTopkThreads;
+  static_assert(kSplitChunk == 2 * kStep, "two sweep steps per chunk");
+  float4 v[2][4];
+#pragma unroll
+  for (int s = 0; s < 2; ++s)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e0 = c0 + s * kStep + 16 * tid + 4 * u;  // rows and chunks are 16-B aligned
+      if (e0 + 3 < c1) {
+        v[s][u] = *reinterpret_cast<const float4*>(row + e0);
+      } else {
+        v[s][u].x = e0 < c1 ? row[e0] : -INFINITY;
+        v[s][u].y = e0 + 1 < c1 ? row[e0 + 1] : -INFINITY;
+        v[s][u].z = e0 + 2 < c1 ? row[e0 + 2] : -INFINITY;
+        v[s][u].w = e0 + 3 < c1 ? row[e0 + 3] : -INFINITY;
+      }
+    }
+  uint32_t* cnt = p.cand_cnt + wrow;
+  uint32_t* ckey = p.cand_key + wrow * kCandCap;
+  int32_t* cpos = p.cand_pos + wrow * kCandCap;
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    const int e0 = c0 + s * kStep + 16 * tid;
+    uint32_t mask = 0;  // bit j: key e0 + j is kept
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      mask |= (v[s][u].x >= thr ? 1u : 0u) << (4 * u);
+      mask |= (v[s][u].y >= thr ? 2u : 0u) << (4 * u);
+      mask |= (v[s][u].z >= thr ? 4u : 0u) << (4 * u);
+      mask |= (v[s][u].w >= thr ? 8u : 0u) << (4 * u);
+    }
+    const int left = c1 - e0;  // -inf past c1 never passes a finite threshold; be exact
+    mask &= left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u);
+    // warp-aggregated append: one atomic per warp reserves the warp's slots
+    const uint32_t c = __popc(mask);
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+    if (tot == 0) continue;  // warp-uniform
+    uint32_t base = 0;
+    if (lane == 31) base = atomicAdd(cnt, tot);
+    base = __shfl_sync(0xffffffffu, base, 31);
+    uint32_t w = base + incl - c;
+    auto put = [&](int j, float x) {
+      if ((mask >> j) & 1u) {
+        if (w < (uint32_t)kCandCap) {
+          ckey[w] = score_key(x);
+          cpos[w] = e0 + j;
+        }
+        ++w;
+      }
+    };
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      put(4 * u, v[s][u].x);
+      put(4 * u + 1, v[s][u].y);
+      put(4 * u + 2, v[s][u].z);
+      put(4 * u + 3, v[s][u].w);
+    }
+  }
+}
+
+constexpr int kSelectSmemBytes =
+    kCandCap * 8 + 2 * kCandMaxWords * 4 + 2048 * 4 + 64 * 4;
+
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_select_kernel(SplitParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(smem_raw);          // [kCandCap]
+  int32_t* cpos = reinterpret_cast<int32_t*>(ckey + kCandCap);     // [kCandCap]
+  float* cache = reinterpret_cast<float*>(smem_raw);               // short rows (<= 8192)
+  uint32_t* sel = reinterpret_cast<uint32_t*>(cpos + kCandCap);    // [kCandMaxWords]
+  uint32_t* tie = sel + kCandMaxWords;                             // [kCandMaxWords]
+  uint32_t* hist = tie + kCandMaxWords;                            // [2048]
+  uint32_t* misc = hist + 2048;                                    // [64]
+  const int64_t wrow = blockIdx.x;
+  const int tid = threadIdx.x;
+  int64_t t;
+  bool ok;
+  const int n = split_row(p, wrow, t, ok);
+  if (n == 0) {  // a bad sequence (reported; its existing rows padded), or no such row
+    const int b = (int)(wrow / p.row_count);
+    const int i = p.row_begin + (int)(wrow - (int64_t)b * p.row_count);
+    if (!ok) {
+      if (tid == 0) report_error(kErrBounds);
+      if (!p.q_start && i < p.q_per_seq)
+        for (int j = tid; j < p.k; j += kTopkThreads) p.idx[t * p.k + j] = -1;
+    }
+    return;
+  }
+  int32_t* out = p.idx + t * p.k;
+  const uint32_t k = (uint32_t)p.k;
+  if (n <= p.k) {
+    for (int j = tid; j < p.k; j += kTopkThreads) out[j] = j < n ? j : -1;
+    return;
+  }
+  const float* row = p.scores + wrow * p.ld;
+  if (n <= 4 * p.k) {
+    select_short_row(row, n, k, cache, hist, misc, out, nullptr);
+    return;
+  }
+  const uint32_t m = p.cand_cnt[wrow];
+  if (m >= k && m <= (uint32_t)kCandCap) {
+    for (uint32_t e = tid; e < m; e += kTopkThreads) {
+      ckey[e] = p.cand_key[wrow * kCandCap + e];
+      cpos[e] = p.cand_pos[wrow * kCandCap + e];
+    }
+    select_from_candidates((int)m, n, k, ckey, cpos, sel, tie, hist, misc, out);
+    return;
+  }
+  // the sample misjudged this row: exact selection over the whole row
   uint32_t tau, r_eq;
-  find_kth((int)m, (uint32_t)p.k, [&](int e, int) { return ckey[e]; }, hist, misc, tau, r_eq);
-  for (uint32_t e = tid; e < m; e += kCandThreads) {
-    const uint32_t key = ckey[e];
-    const int pos = cpos[e];
-    if (key > tau) atomicOr(&sel[pos >> 5], 1u << (pos & 31));
-    else if (key == tau) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
-  }
-  __syncthreads();
-  // the r_eq lowest positions among the keys equal to tau: an ordered scan of the
-  // tie bitmap (each thread owns consecutive words)
-  const int per = (words + kCandThreads - 1) / kCandThreads;
-  const int w0 = tid * per;
-  uint32_t cnt = 0;
-  for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(tie[w]);
-  uint32_t before = block_exclusive_scan(cnt, misc, misc + 32);
-  for (int w = w0; w < w0 + per && w < words; ++w) {
-    uint32_t bits = tie[w];
-    while (bits) {
-      const uint32_t bit = bits & (~bits + 1u);
-      if (before < r_eq) sel[w] |= bit;
-      ++before;
-      bits ^= bit;
-    }
-  }
-  __syncthreads();
-  // ascending compaction of the selection (exactly k marks)
-  cnt = 0;
-  for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(sel[w]);
-  uint32_t o = block_exclusive_scan(cnt, misc, misc + 32);
-  for (int w = w0; w < w0 + per && w < words; ++w) {
-    uint32_t bits = sel[w];
-    while (bits) {
-      const int bpos = __ffs(bits) - 1;
-      if (o < (uint32_t)p.k) out[o] = w * 32 + bpos;
-      ++o;
-      bits &= bits - 1u;
-    }
-  }
+  find_kth(n, k, [&](int e, int) { return score_key(row[e]); }, hist, misc, tau, r_eq);
+  compact_topk(n, tau, r_eq, [&](int e, int) { return score_key(row[e]); },
+               [&](int e) { return e; }, out, misc);
 }
 
 }  // namespace dsa

@@ -59,6 +59,11 @@ SIGNATURES = {
                                           ctypes.POINTER(QDescC), _P, ctypes.c_int64, _P]),
     "dsa_topk": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.POINTER(KvDescC),
                                 ctypes.POINTER(QDescC), ctypes.c_int32, _P, _P]),
+    "dsa_topk_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
+                                                  ctypes.c_int32]),
+    "dsa_topk_ws": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.POINTER(KvDescC),
+                                   ctypes.POINTER(QDescC), ctypes.c_int32, _P, ctypes.c_size_t,
+                                   _P, _P]),
     "dsa_sparse_mla_fwd": (ctypes.c_int, [_P, _P, ctypes.POINTER(KvDescC), ctypes.POINTER(QDescC),
                                           _P, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "dsa_sparse_mla_fwd_ws": (ctypes.c_int, [_P, _P, ctypes.POINTER(KvDescC),
@@ -228,6 +233,40 @@ def dsa_topk(scores, kv: KvLayout, q_per_seq: int, k: int,
     kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
     _check(lib().dsa_topk(_ptr(scores), scores.shape[1], ctypes.byref(kvd), ctypes.byref(qd), k,
                           _ptr(idx), _stream(stream)), "dsa_topk")
+    return idx
+
+
+def dsa_topk_workspace_size(kv: KvLayout, num_q: int, q_per_seq: int, k: int, rows=None,
+                            q_start=None) -> int:
+    kvd, qd = kv.c(), _qdesc(num_q, q_per_seq, rows, q_start)
+    return int(lib().dsa_topk_workspace_size(ctypes.byref(kvd), ctypes.byref(qd), k))
+
+
+def dsa_topk_ws(scores, kv: KvLayout, q_per_seq: int, k: int, workspace=None,
+                idx: Optional[torch.Tensor] = None, rows=None, stream=None, q_start=None,
+                num_q: Optional[int] = None) -> torch.Tensor:
+    """dsa_topk with scratch for sweeping long rows with several CTAs (include/dsa.h);
+    ``workspace`` is a 256-B aligned device tensor (a fresh one of
+    dsa_topk_workspace_size() bytes when None). Same selection as dsa_topk."""
+    if q_start is None:
+        T = kv.batch * q_per_seq
+    elif num_q is not None:
+        T = num_q
+    elif idx is not None:
+        T = idx.shape[0]
+    else:
+        raise ValueError("dsa_topk_ws on a ragged batch needs idx or num_q")
+    if idx is None:
+        idx = torch.empty(T, k, dtype=torch.int32, device=scores.device)
+    if workspace is None:
+        workspace = torch.empty(max(256, dsa_topk_workspace_size(kv, T, q_per_seq, k, rows,
+                                                                 q_start)),
+                                dtype=torch.uint8, device=scores.device)
+    kvd, qd = kv.c(), _qdesc(T, q_per_seq, rows, q_start)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().dsa_topk_ws(_ptr(scores), scores.shape[1], ctypes.byref(kvd), ctypes.byref(qd),
+                             k, _ptr(workspace), nbytes, _ptr(idx), _stream(stream)),
+           "dsa_topk_ws")
     return idx
 
 

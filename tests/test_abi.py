@@ -137,14 +137,29 @@ def test_host_argument_checks_without_gpu(lib):
 def test_workspace_size_plan(lib):
     from sparse_attention_05_b200 import dsa
     by = ctypes.byref
-    # decode, 64 x 32768: indices + all score rows in one chunk
+    def split(rows):  # the split top-k's candidates (8192 keys + positions), counts, thresholds
+        return rows * 8192 * 8 + 2 * ((rows * 4 + 255) // 256 * 256)
+    # decode, 64 x 32768: indices + all score rows in one chunk (the forward's top-k
+    # is one CTA per row); dsa_topk_ws's split scratch on its own
     kv, q = _kv(batch=64, max_ctx=32768), dsa.QDescC(64, 1, 0, 0)
     n = lib.dsa_workspace_size(by(kv), by(q), 2048)
     assert n == 64 * 2048 * 4 + 64 * 32768 * 4
-    # prefill 131072: indices + one 2 GiB chunk of score rows
+    assert lib.dsa_topk_workspace_size(by(kv), by(q), 2048) == split(64)
+    # prefill 131072: indices + one 2 GiB chunk of score rows (many rows: no split top-k)
     kv, q = _kv(batch=1, max_ctx=131072), dsa.QDescC(131072, 131072, 0, 0)
     n = lib.dsa_workspace_size(by(kv), by(q), 2048)
     assert n == 131072 * 2048 * 4 + 4096 * 131072 * 4
+    assert lib.dsa_topk_workspace_size(by(kv), by(q), 2048) == 0
+    # 4 x 148 rows still split, one more does not
+    kv = _kv(batch=592, max_ctx=65536)
+    assert lib.dsa_topk_workspace_size(by(kv), by(dsa.QDescC(592, 1, 0, 0)), 2048) == split(592)
+    kv = _kv(batch=593, max_ctx=65536)
+    assert lib.dsa_topk_workspace_size(by(kv), by(dsa.QDescC(593, 1, 0, 0)), 2048) == 0
+    # rows no longer than 4k keys, or longer than the selection bitmaps: no split
+    kv, q = _kv(batch=4, max_ctx=8192), dsa.QDescC(4, 1, 0, 0)
+    assert lib.dsa_topk_workspace_size(by(kv), by(q), 2048) == 0
+    kv, q = _kv(batch=1, max_ctx=131073), dsa.QDescC(1, 1, 0, 0)
+    assert lib.dsa_topk_workspace_size(by(kv), by(q), 2048) == 0
     # invalid geometry -> 0
     assert lib.dsa_workspace_size(by(kv), by(dsa.QDescC(5, 131072, 0, 0)), 2048) == 0
 

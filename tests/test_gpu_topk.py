@@ -17,16 +17,22 @@ def _dsa():
 
 
 def _run(scores_np, seqlens, q_per_seq, k):
+    """dsa_topk (one CTA per row) and dsa_topk_ws (long rows split across CTAs) on
+    the same rows: both must equal the oracle's selection; returns the one-CTA
+    result (and checks the split one inside)."""
     dsa = _dsa()
     T, ld = scores_np.shape
     B = len(seqlens)
     kv = dsa.KvLayout(batch=B, max_ctx=ld,
                       seqlens=torch.tensor(seqlens, dtype=torch.int32, device="cuda"))
-    idx = dsa.dsa_topk(torch.from_numpy(scores_np).cuda(), kv, q_per_seq, k)
+    s = torch.from_numpy(scores_np).cuda()
+    idx = dsa.dsa_topk(s, kv, q_per_seq, k)
+    idx_split = dsa.dsa_topk_ws(s, kv, q_per_seq, k)
     torch.cuda.synchronize()
     assert dsa.dsa_get_device_error() == 0
     pos = np.array([seqlens[t // q_per_seq] - q_per_seq + t % q_per_seq for t in range(T)])
     want = topk_rows(scores_np, pos, k)
+    np.testing.assert_array_equal(idx_split.cpu().numpy(), want)
     return idx.cpu().numpy(), want
 
 
@@ -91,4 +97,34 @@ def test_masked_tail_is_never_read():
     s[0, 5000:] = np.inf  # beyond pos: must be ignored
     s[1, 3000:] = np.nan
     got, want = _run(s, [5000, 3000], 1, 2048)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_split_rows_whose_sample_misjudges_take_the_full_row_path():
+    """Rows built so that the strided sample's threshold is useless: the sampled
+    positions hold the row's largest scores (fewer than k candidates pass), or its
+    smallest (nearly every key passes, more than the candidate list holds). The
+    split selection must still be exact (it falls back to the whole row)."""
+    rng = np.random.default_rng(11)
+    n = 131072
+    rows = np.empty((3, n), np.float32)
+    sampled = (np.arange(2048, dtype=np.int64) * n) // 2048
+    rows[0] = rng.standard_normal(n).astype(np.float32)
+    rows[0][sampled] = 100.0 + rng.random(2048).astype(np.float32)  # threshold too high
+    rows[1] = 10.0 + rng.random(n).astype(np.float32)
+    rows[1][sampled] = -100.0                                         # threshold too low
+    rows[2] = rng.standard_normal(n).astype(np.float32)               # a plain row
+    got, want = _run(rows, [n, n, 70001], 1, 2048)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_split_chunk_edges_and_hot_ties():
+    """Rows whose lengths end just past, at and before chunk edges (16384 keys), with
+    the top scores tied across chunk boundaries."""
+    rng = np.random.default_rng(12)
+    ld = 65536
+    seqlens = [16384, 16385, 32767, 8193, 49153, 65536]
+    s = (rng.integers(0, 40, (len(seqlens), ld)) / 8.0).astype(np.float32)
+    s[:, 16380:16390] = 9.0  # ties straddling the first chunk edge
+    got, want = _run(s, seqlens, 1, 2048)
     np.testing.assert_array_equal(got, want)
