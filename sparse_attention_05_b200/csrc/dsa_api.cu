@@ -155,21 +155,19 @@ size_t split_topk_bytes(int64_t rows) {
   return align256((size_t)rows * kCandCap * 8) + 2 * align256((size_t)rows * 4);
 }
 
-// Whether the split path applies: some row may hold more than 4k keys (else the
-// one-CTA kernel has nothing to split), every row fits the selection bitmaps, and
-// the rows are few enough that one CTA per row would leave SMs idle (with many rows,
-// as in prefill, every SM is busy anyway and splitting only adds launches).
 // dsa_forward's choice between the two selections. Measured on B200 (paged 128K
-// decode, 256 rows): the split path's threshold, sweep and select kernels take 16 +
-// 36 + 28 us against 78 us for one CTA per row (each of the three is bound by fixed
-// latency: short-lived sweep CTAs in waves, and the block-wide radix passes of the
-// threshold and of the selection), so the forward keeps one CTA per row; the split
-// path stays available through dsa_topk_ws.
+// decode, 256 rows, CUDA events around the selection inside the step): the split
+// path takes 98 us (its threshold, sweep and select kernels share it about 21 : 50 :
+// 29) against 78 us for one CTA per row. Each of the three is bound by fixed latency
+// (short-lived sweep CTAs in waves, and the block-wide radix passes of the threshold
+// and of the selection), so the forward keeps one CTA per row; the split path stays
+// available through dsa_topk_ws.
 constexpr bool kForwardSplitTopk = false;
 
+// Whether the split path applies: some row may hold more than 4k keys (else the
+// one-CTA kernel has nothing to split) and every row fits the selection bitmaps.
 bool split_topk_applies(const Geometry& g, int k) {
-  return g.max_ctx > 4 * k && g.max_ctx <= kCandMaxWords * 32 &&
-         (int64_t)g.batch * g.row_count <= 4 * (int64_t)num_sms();
+  return g.max_ctx > 4 * k && g.max_ctx <= kCandMaxWords * 32;
 }
 
 dsa_status_t launch_topk_split(const float* scores, int64_t ld, const Geometry& g,
@@ -177,13 +175,8 @@ dsa_status_t launch_topk_split(const float* scores, int64_t ld, const Geometry& 
                                cudaStream_t stream, void* scratch) {
   static DeviceOnce once;
   const cudaError_t attr_err = once_per_device(once, [] {
-    cudaError_t e = cudaFuncSetAttribute(topk_threshold_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kThresholdSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kSelectSmemBytes);
-    return e;
+    return cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kSelectSmemBytes);
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
   const int64_t rows = (int64_t)g.batch * row_count;
@@ -208,7 +201,7 @@ dsa_status_t launch_topk_split(const float* scores, int64_t ld, const Geometry& 
   p.thr_key = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.cand_cnt) +
                                           align256((size_t)rows * 4));
   p.idx = idx;
-  topk_threshold_kernel<<<(unsigned)rows, kTopkThreads, kThresholdSmemBytes, stream>>>(p);
+  topk_threshold_kernel<<<(unsigned)rows, kThresholdThreads, 0, stream>>>(p);
   dsa_status_t st = cuda_status(cudaGetLastError());
   if (st != DSA_OK) return st;
   topk_sweep_kernel<<<(unsigned)(rows * p.nchunk), kTopkThreads, 0, stream>>>(p);
@@ -269,6 +262,9 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(indexer_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kIdxSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(indexer_kernel<false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmemBytes);
     return e;
   });
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
@@ -278,6 +274,8 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   if (st != DSA_OK) return st;
   IndexerParams p{};
   p.q_idx = reinterpret_cast<const __nv_bfloat16*>(q_idx);
+  p.k_idx = reinterpret_cast<const uint8_t*>(k_idx);
+  p.cache_rows = g.cache_rows;
   p.w = w;
   p.k_scale = k_scale;
   p.block_table = g.block_table;
@@ -310,6 +308,9 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   const int grid = (int)std::min<int64_t>(max_tiles, num_sms());
   if (p.thr) {
     indexer_kernel<true><<<grid, kIdxThreads, kIdxSmemBytes, stream>>>(p, tm);
+  } else if (p.paged && p.G <= 2) {
+    // paged decode: the copy warps take half of each tile's 8-KB random-page reads
+    indexer_kernel<false, true><<<grid, kIdxAssistThreads, kIdxSmemBytes, stream>>>(p, tm);
   } else {
     indexer_kernel<false><<<grid, kIdxThreads, kIdxSmemBytes, stream>>>(p, tm);
   }

@@ -44,6 +44,11 @@ constexpr int kIdxDim = 128;
 constexpr int kIdxTile = 128;                      // keys per tile (MMA M)
 constexpr int kIdxStages = 8;
 constexpr int kIdxThreads = 384;
+// Paged decode form: four more warps (12-15) bring the second half of every key tile
+// with cp.async beside the producer's TMA box (see indexer_kernel's kAssist).
+constexpr int kIdxAssistThreads = 512;
+constexpr int kIdxCpWarp0 = 12;
+constexpr int kIdxCpThreads = 128;
 constexpr int kIdxStageBytes = kIdxTile * kIdxDim;  // 16 KB of e4m3
 constexpr int kIdxQBufBytes = 4 * kIdxHeads * kIdxDim;  // G <= 4 rows x 64 heads x 128 B
 constexpr int kIdxSmemBytes =
@@ -54,6 +59,8 @@ constexpr int kIdxMaxAcc = 8;  // TMEM accumulators: 512 / N, at most 8
 
 struct IndexerParams {
   const __nv_bfloat16* q_idx;  // [T][64][128]
+  const uint8_t* k_idx;        // [cache_rows][128] E4M3 key codes (the copy warps' half tiles)
+  int64_t cache_rows;
   const float* w;              // [T][64]
   const float* k_scale;        // [cache_rows]
   const int32_t* block_table;  // [batch][max_pages] when paged
@@ -209,10 +216,18 @@ __device__ void idx_share(const IndexerParams& p, IdxShare* out, uint32_t* scrat
 
 // kFilter: the fused selection's filter mode (thr, cand_* set; no score rows); the
 // plain instantiation carries none of its code.
-template <bool kFilter>
-__global__ void __launch_bounds__(kIdxThreads, 1)
+// kAssist (paged caches, at most 2 query rows per group): each key tile arrives as one
+// TMA box of 64 keys (the producer) and 64 keys copied in 16-B cp.async pieces by four
+// extra warps. A per-SM trace of the paged decode showed the producer's TMA issue
+// holding only about two tiles in flight (one 8-KB random-page box per ~800 cycles),
+// so the tile stream was bound by the TMA unit; the copy warps take half of it. The
+// 16 warps leave 128 registers per thread, so the epilogue reads tensor memory in
+// 16-column chunks.
+template <bool kFilter, bool kAssist = false>
+__global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ IndexerParams p,
                    const __grid_constant__ CUtensorMap tm_keys) {
+  static_assert(!(kFilter && kAssist), "the copy-assisted form is for plain scores");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -244,7 +259,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kIdxStages; ++s) {
-      mbar_init(smem_u32(&kfull[s]), 1);   // expect_tx arrival (+ the tile's bytes)
+      // expect_tx arrival (+ the TMA bytes), and one arrival per copy thread
+      mbar_init(smem_u32(&kfull[s]), kAssist ? 1 + kIdxCpThreads : 1);
       mbar_init(smem_u32(&kempty[s]), 1);  // the MMA's commit
     }
     for (int i = 0; i < kIdxMaxAcc; ++i) {
@@ -321,9 +337,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           }
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(bar, kIdxStageBytes);
+          mbar_arrive_expect_tx(bar, kAssist ? kIdxStageBytes / 2 : kIdxStageBytes);
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
+          for (int h = 0; h < (kAssist ? 1 : 2); ++h)  // kAssist: keys 64-127 by the copy warps
             tma_load_2d(smem_u32(stages + st * kIdxStageBytes + h * 8192), &tm_keys, bar, 0,
                         (int)base[h]);
         }
@@ -355,6 +371,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             break;
           }
           tc_fence_after();
+          if (kAssist) fence_proxy_async_smem();  // cp.async (generic proxy) -> tensor core
           const uint32_t kaddr = smem_u32(stages + st * kIdxStageBytes);
           const uint32_t dcol = tmem_base + ab * N;
 #pragma unroll
@@ -375,6 +392,50 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       mbar_wait(smem_u32(mdone), 0, TO, no_abort);
     }
     __syncwarp();
+  } else if (kAssist && warp >= kIdxCpWarp0) {
+    // ------------------------------------------------------------ cp.async copy warps
+    // Keys 64-127 of each tile (64 rows x 128 B) in 16-B pieces, four per thread,
+    // written in the 128-B swizzled layout the TMA gives the first half; each thread
+    // arrives on the stage barrier once its pieces have landed. Rows past the cache
+    // end (a contiguous cache whose length is not a multiple of 128) read as zeros.
+    const int ct = tid - kIdxCpWarp0 * 32;
+    uint32_t it = 0;
+    IdxCursor cur{sh.gs, sh.ts};
+    IdxUnit U;
+    bool ok = true;
+    while (ok && !*abort_flag && idx_next(p, sh, cur, U)) {
+      const int pos_max = U.seqlen - U.q_len + U.i0 + U.nrows - 1;
+      for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
+        const int st = it % kIdxStages;
+        if (!warp_wait(smem_u32(&kempty[st]), ((it / kIdxStages) & 1) ^ 1, TO, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int s0 = kt * p.tile_stride * kIdxTile + 64;
+        int64_t base = 0;  // past pos_max or behind a bad page: row 0 (masked later)
+        if (s0 <= pos_max) {
+          if (!p.paged) {
+            base = (int64_t)U.b * p.max_ctx + s0;
+          } else {
+            const int page = __ldg(p.block_table + (int64_t)U.b * p.max_pages + s0 / p.page_size);
+            if (page >= 0 && page < p.num_pages)
+              base = (int64_t)page * p.page_size + s0 % p.page_size;
+          }
+        }
+        const uint8_t* src = p.k_idx + base * kIdxDim;
+        const uint32_t dst = smem_u32(stages + st * kIdxStageBytes + 8192);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = ct + kIdxCpThreads * i;  // piece: row c / 8, 16-B column c % 8
+          const int r = c >> 3, j = c & 7;
+          const bool in = base + r < p.cache_rows;
+          cp_async_16(dst + r * 128 + ((j ^ (r & 7)) << 4), in ? src + r * 128 + j * 16 : p.k_idx,
+                      in ? 16u : 0u);
+        }
+        cp_async_mbar_arrive(smem_u32(&kfull[st]));
+      }
+    }
+    cp_async_wait_all();
   } else if (warp < 4) {
     // ------------------------------------------------------------ query quantizers
     const int qw = warp - 2;  // 0..1
@@ -514,35 +575,11 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           break;
         }
         tc_fence_after();
-        // Row gi's 64 head columns come as two 32-column chunks (A: heads
-        // 0-31, B: heads 32-63). The next chunk's load is always in flight
-        // while the current one is reduced, so the tensor-memory load latency
-        // hides behind the ReLU / weighted head sum.
         const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) + ab * N;
-        uint32_t ca[32], cb[32];
         uint32_t take_bits = 0;  // filter mode: rows that keep this thread's key
-        tmem_ld32u(tcol, ca);
-        tmem_wait_ld_fence(ca);
-        for (int gi = 0; gi < U.nrows; ++gi) {
-          const float4* w4 = reinterpret_cast<const float4*>(wrow + gi * kIdxHeads);
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-          auto reduce32 = [&](const uint32_t (&v)[32], const float4* wq4) {
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const float4 wv = wq4[q4];
-              a0 = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * q4 + 0]), 0.f), a0);
-              a1 = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * q4 + 1]), 0.f), a1);
-              a2 = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * q4 + 2]), 0.f), a2);
-              a3 = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * q4 + 3]), 0.f), a3);
-            }
-          };
-          tmem_ld32u(tcol + gi * kIdxHeads + 32, cb);
-          reduce32(ca, w4);
-          tmem_wait_ld_fence(cb);
-          if (gi + 1 < U.nrows) tmem_ld32u(tcol + (gi + 1) * kIdxHeads, ca);
-          reduce32(cb, w4 + 8);
-          if (gi + 1 < U.nrows) tmem_wait_ld_fence(ca);
-          const float acc = (a0 + a1) + (a2 + a3);
+        // row gi's score from its weighted head sum: causal mask, key scale, then the
+        // score row (or, in filter mode, the candidate note)
+        auto finish_row = [&](int gi, float acc) {
           const float out = (s <= pos0 + gi) ? ks * acc : -INFINITY;
           const int64_t orow = (int64_t)U.b * p.row_count + (U.i0 - p.row_begin) + gi;
           if (!kFilter) {
@@ -551,6 +588,70 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             const bool take = s <= pos0 + gi && out >= thr_row[gi];
             take_bits |= (take ? 1u : 0u) << gi;
             cstage[((cpar * 4 + gi) << 8) + et] = score_key(out);
+          }
+        };
+        if constexpr (kAssist) {
+          // 16-column chunks (the 16-warp form's register budget): row gi's 64 head
+          // columns as four chunks, the next one's load in flight while one is reduced
+          uint32_t ca[16], cb[16];
+          tmem_ld16u(tcol, ca);
+          tmem_wait_ld_fence16(ca);
+          for (int gi = 0; gi < U.nrows; ++gi) {
+            const float4* w4 = reinterpret_cast<const float4*>(wrow + gi * kIdxHeads);
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            auto reduce16 = [&](const uint32_t (&v)[16], const float4* wq4) {
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 wv = wq4[q4];
+                a0 = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * q4 + 0]), 0.f), a0);
+                a1 = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * q4 + 1]), 0.f), a1);
+                a2 = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * q4 + 2]), 0.f), a2);
+                a3 = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * q4 + 3]), 0.f), a3);
+              }
+            };
+            const uint32_t rc = tcol + gi * kIdxHeads;
+            tmem_ld16u(rc + 16, cb);
+            reduce16(ca, w4);
+            tmem_wait_ld_fence16(cb);
+            tmem_ld16u(rc + 32, ca);
+            reduce16(cb, w4 + 4);
+            tmem_wait_ld_fence16(ca);
+            tmem_ld16u(rc + 48, cb);
+            reduce16(ca, w4 + 8);
+            tmem_wait_ld_fence16(cb);
+            if (gi + 1 < U.nrows) tmem_ld16u(tcol + (gi + 1) * kIdxHeads, ca);
+            reduce16(cb, w4 + 12);
+            if (gi + 1 < U.nrows) tmem_wait_ld_fence16(ca);
+            finish_row(gi, (a0 + a1) + (a2 + a3));
+          }
+        } else {
+          // Row gi's 64 head columns come as two 32-column chunks (A: heads 0-31, B:
+          // heads 32-63). The next chunk's load is always in flight while the current
+          // one is reduced, so the tensor-memory load latency hides behind the ReLU /
+          // weighted head sum.
+          uint32_t ca[32], cb[32];
+          tmem_ld32u(tcol, ca);
+          tmem_wait_ld_fence(ca);
+          for (int gi = 0; gi < U.nrows; ++gi) {
+            const float4* w4 = reinterpret_cast<const float4*>(wrow + gi * kIdxHeads);
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            auto reduce32 = [&](const uint32_t (&v)[32], const float4* wq4) {
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4) {
+                const float4 wv = wq4[q4];
+                a0 = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * q4 + 0]), 0.f), a0);
+                a1 = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * q4 + 1]), 0.f), a1);
+                a2 = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * q4 + 2]), 0.f), a2);
+                a3 = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * q4 + 3]), 0.f), a3);
+              }
+            };
+            tmem_ld32u(tcol + gi * kIdxHeads + 32, cb);
+            reduce32(ca, w4);
+            tmem_wait_ld_fence(cb);
+            if (gi + 1 < U.nrows) tmem_ld32u(tcol + (gi + 1) * kIdxHeads, ca);
+            reduce32(cb, w4 + 8);
+            if (gi + 1 < U.nrows) tmem_wait_ld_fence(ca);
+            finish_row(gi, (a0 + a1) + (a2 + a3));
           }
         }
         tc_fence_before();

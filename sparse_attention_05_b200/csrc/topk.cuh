@@ -545,59 +545,96 @@ __device__ __forceinline__ int split_row(const SplitParams& p, int64_t wrow, int
   return R.seqlen - R.q_len + i + 1;
 }
 
-// Threshold key of a long row: the r-th largest of the fixed strided sample of 2048
-// scores, r = expected count of top-k keys in the sample + 4 standard deviations + 16
-// (the same threshold the one-CTA path of topk_kernel uses).
-__device__ __forceinline__ uint32_t long_row_threshold(const float* row, int n, uint32_t k,
-                                                       uint32_t* sample, uint32_t* hist,
-                                                       uint32_t* misc) {
-  for (int s = threadIdx.x; s < kTopkSample; s += kTopkThreads)
-    sample[s] = score_key(row[(int64_t)s * n / kTopkSample]);
-  __syncthreads();
-  const float expect = (float)k / (float)n * kTopkSample;
-  uint32_t r = (uint32_t)(expect + 4.0f * sqrtf(expect) + 16.0f);
-  r = min(r, (uint32_t)kTopkSample);
-  uint32_t tau_low, unused;
-  find_kth(kTopkSample, r, [&](int e, int) { return sample[e]; }, hist, misc, tau_low, unused);
-  return tau_low;
-}
+// Threshold key of a long row, the one topk_kernel's one-CTA path uses: the r-th
+// largest of the fixed strided sample of 2048 scores, r = the expected count of top-k
+// keys in the sample + 4 standard deviations + 16. One CTA of 4 warps per row computes
+// it: each thread holds 16 sampled keys, and four passes over 8-bit digits (a
+// 256-bin histogram with match.any-aggregated shared atomics, then a scan of the bins
+// by warp 0) narrow the prefix down to the exact key.
+constexpr int kThresholdThreads = 128;
 
-constexpr int kThresholdSmemBytes = 2048 * 4 + 64 * 4 + kTopkSample * 4;
+__device__ __forceinline__ uint32_t sample_threshold(const float* row, int n, uint32_t k,
+                                                     uint32_t* hist, uint32_t* bcast) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kPer = kTopkSample / kThresholdThreads;  // 16 sampled keys per thread
+  uint32_t key[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j)
+    key[j] = score_key(row[(int64_t)(tid + kThresholdThreads * j) * n / kTopkSample]);
+  const float expect = (float)k / (float)n * kTopkSample;
+  uint32_t remaining = (uint32_t)(expect + 4.0f * sqrtf(expect) + 16.0f);
+  remaining = min(remaining, (uint32_t)kTopkSample);
+  uint32_t prefix = 0, mask = 0;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = tid; b < 256; b += kThresholdThreads) hist[b] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const uint32_t digit = (key[j] & mask) == prefix ? (key[j] >> shift) & 255u : 256u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+      if (digit < 256u && (__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], __popc(peers));
+    }
+    __syncthreads();
+    if (warp == 0) {  // bins from the top: lane l owns bins 255 - 8 l - i, i < 8
+      uint32_t cnt[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cnt[i] = hist[255 - 8 * lane - i];
+        sum += cnt[i];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+      }
+      uint32_t above = incl - sum;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (above < remaining && remaining <= above + cnt[i]) {  // exactly one (lane, i)
+          bcast[0] = 255u - 8u * lane - i;
+          bcast[1] = remaining - above;
+        }
+        above += cnt[i];
+      }
+    }
+    __syncthreads();
+    prefix |= bcast[0] << shift;
+    mask |= 255u << shift;
+    remaining = bcast[1];
+  }
+  return prefix;
+}
 
 // One CTA per window row: zeroes the row's candidate count and, for a long row,
 // computes its threshold key once for all of its chunk CTAs.
-__global__ void __launch_bounds__(kTopkThreads, 2) topk_threshold_kernel(SplitParams p) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
-  uint32_t* misc = hist + 2048;
-  uint32_t* sample = misc + 64;
+__global__ void __launch_bounds__(kThresholdThreads) topk_threshold_kernel(SplitParams p) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t bcast[2];
   const int64_t wrow = blockIdx.x;
   int64_t t;
   bool ok;
   const int n = split_row(p, wrow, t, ok);
   if (threadIdx.x == 0) p.cand_cnt[wrow] = 0u;
   if (n <= 4 * p.k) return;
-  const uint32_t thr =
-      long_row_threshold(p.scores + wrow * p.ld, n, (uint32_t)p.k, sample, hist, misc);
+  const uint32_t thr = sample_threshold(p.scores + wrow * p.ld, n, (uint32_t)p.k, hist, bcast);
   if (threadIdx.x == 0) p.thr_key[wrow] = thr;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 2) topk_sweep_kernel(SplitParams p) {
-  const int64_t wrow = blockIdx.x / p.nchunk;
-  const int chunk = (int)(blockIdx.x - wrow * p.nchunk);
-  int64_t t;
-  bool ok;
-  const int n = split_row(p, wrow, t, ok);
-  const int c0 = chunk * kSplitChunk;
-  if (n <= 4 * p.k || c0 >= n) return;  // short rows and chunks past the row: no sweep
-  const int c1 = min(n, c0 + kSplitChunk);
-  const float* row = p.scores + wrow * p.ld;
-  const float thr = key_score(p.thr_key[wrow]);
-  // 16 consecutive keys per thread per step (8192 keys), both steps' loads issued
-  // before either is used; keys >= thr <=> key >= threshold key (no NaN scores)
-  const int tid = threadIdx.x, lane = tid & 31;
+// Sweep of keys [c0, c1) of a long row (c1 - c0 <= kSplitChunk, c0 a multiple of 16):
+// 16 consecutive keys per thread per step (8192 keys), both steps' loads issued before
+// either is used; keys with a score >= thr (<=> key >= the threshold key: no NaN
+// scores) are appended to the row's list. The CTA reserves its slots with one atomic
+// for the whole chunk (a block scan of the threads' counts: every chunk CTA of a row
+// adds to the same counter, so per-warp atomics would queue at one address); slots
+// past kCandCap are counted but not written. `scan` is 32 words of shared memory.
+__device__ __forceinline__ void sweep_chunk(const float* row, int c0, int c1, float thr,
+                                            uint32_t* cnt, uint32_t* ckey, int32_t* cpos,
+                                            uint32_t* scan) {
   constexpr int kStep = 16 * kTopkThreads;
   static_assert(kSplitChunk == 2 * kStep, "two sweep steps per chunk");
+  const int tid = threadIdx.x;
   float4 v[2][4];
 #pragma unroll
   for (int s = 0; s < 2; ++s)
@@ -613,38 +650,30 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_sweep_kernel(SplitParams
         v[s][u].w = e0 + 3 < c1 ? row[e0 + 3] : -INFINITY;
       }
     }
-  uint32_t* cnt = p.cand_cnt + wrow;
-  uint32_t* ckey = p.cand_key + wrow * kCandCap;
-  int32_t* cpos = p.cand_pos + wrow * kCandCap;
+  uint32_t mask[2];  // bit j of mask[s]: key c0 + s kStep + 16 tid + j is kept
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      m |= (v[s][u].x >= thr ? 1u : 0u) << (4 * u);
+      m |= (v[s][u].y >= thr ? 2u : 0u) << (4 * u);
+      m |= (v[s][u].z >= thr ? 4u : 0u) << (4 * u);
+      m |= (v[s][u].w >= thr ? 8u : 0u) << (4 * u);
+    }
+    const int left = c1 - (c0 + s * kStep + 16 * tid);  // -inf past c1 never passes; be exact
+    mask[s] = m & (left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u));
+  }
+  const uint32_t mine = __popc(mask[0]) + __popc(mask[1]);
+  const uint32_t before = block_exclusive_scan(mine, scan, scan + 16);
+  if (tid == 0 && scan[16] > 0u) scan[17] = atomicAdd(cnt, scan[16]);
+  __syncthreads();
+  uint32_t w = scan[17] + before;
 #pragma unroll
   for (int s = 0; s < 2; ++s) {
     const int e0 = c0 + s * kStep + 16 * tid;
-    uint32_t mask = 0;  // bit j: key e0 + j is kept
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      mask |= (v[s][u].x >= thr ? 1u : 0u) << (4 * u);
-      mask |= (v[s][u].y >= thr ? 2u : 0u) << (4 * u);
-      mask |= (v[s][u].z >= thr ? 4u : 0u) << (4 * u);
-      mask |= (v[s][u].w >= thr ? 8u : 0u) << (4 * u);
-    }
-    const int left = c1 - e0;  // -inf past c1 never passes a finite threshold; be exact
-    mask &= left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u);
-    // warp-aggregated append: one atomic per warp reserves the warp's slots
-    const uint32_t c = __popc(mask);
-    uint32_t incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += x;
-    }
-    const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
-    if (tot == 0) continue;  // warp-uniform
-    uint32_t base = 0;
-    if (lane == 31) base = atomicAdd(cnt, tot);
-    base = __shfl_sync(0xffffffffu, base, 31);
-    uint32_t w = base + incl - c;
     auto put = [&](int j, float x) {
-      if ((mask >> j) & 1u) {
+      if ((mask[s] >> j) & 1u) {
         if (w < (uint32_t)kCandCap) {
           ckey[w] = score_key(x);
           cpos[w] = e0 + j;
@@ -660,6 +689,23 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_sweep_kernel(SplitParams
       put(4 * u + 3, v[s][u].w);
     }
   }
+  __syncthreads();  // scan[] is reused by the CTA's next chunk
+}
+
+// One CTA per (row, chunk); a CTA whose row is short or whose chunk lies past the row
+// exits at once.
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_sweep_kernel(SplitParams p) {
+  __shared__ uint32_t scan[32];
+  const int64_t wrow = blockIdx.x / p.nchunk;
+  const int chunk = (int)(blockIdx.x - wrow * p.nchunk);
+  int64_t t;
+  bool ok;
+  const int n = split_row(p, wrow, t, ok);
+  const int c0 = chunk * kSplitChunk;
+  if (n <= 4 * p.k || c0 >= n) return;  // short rows and chunks past the row: no sweep
+  const int c1 = min(n, c0 + kSplitChunk);
+  sweep_chunk(p.scores + wrow * p.ld, c0, c1, key_score(p.thr_key[wrow]), p.cand_cnt + wrow,
+              p.cand_key + wrow * kCandCap, p.cand_pos + wrow * kCandCap, scan);
 }
 
 constexpr int kSelectSmemBytes =

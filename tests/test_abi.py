@@ -145,16 +145,13 @@ def test_workspace_size_plan(lib):
     n = lib.dsa_workspace_size(by(kv), by(q), 2048)
     assert n == 64 * 2048 * 4 + 64 * 32768 * 4
     assert lib.dsa_topk_workspace_size(by(kv), by(q), 2048) == split(64)
-    # prefill 131072: indices + one 2 GiB chunk of score rows (many rows: no split top-k)
+    # prefill 131072: indices + one 2 GiB chunk of score rows
     kv, q = _kv(batch=1, max_ctx=131072), dsa.QDescC(131072, 131072, 0, 0)
     n = lib.dsa_workspace_size(by(kv), by(q), 2048)
     assert n == 131072 * 2048 * 4 + 4096 * 131072 * 4
-    assert lib.dsa_topk_workspace_size(by(kv), by(q), 2048) == 0
-    # 4 x 148 rows still split, one more does not
-    kv = _kv(batch=592, max_ctx=65536)
-    assert lib.dsa_topk_workspace_size(by(kv), by(dsa.QDescC(592, 1, 0, 0)), 2048) == split(592)
-    kv = _kv(batch=593, max_ctx=65536)
-    assert lib.dsa_topk_workspace_size(by(kv), by(dsa.QDescC(593, 1, 0, 0)), 2048) == 0
+    # dsa_topk_ws's scratch for one 4096-row window of it
+    q = dsa.QDescC(131072, 131072, 0, 4096)
+    assert lib.dsa_topk_workspace_size(by(kv), by(q), 2048) == split(4096)
     # rows no longer than 4k keys, or longer than the selection bitmaps: no split
     kv, q = _kv(batch=4, max_ctx=8192), dsa.QDescC(4, 1, 0, 0)
     assert lib.dsa_topk_workspace_size(by(kv), by(q), 2048) == 0
