@@ -157,8 +157,8 @@ size_t split_topk_bytes(int64_t rows) {
 
 // dsa_forward's choice between the two selections. Measured on B200 (paged 128K
 // decode, 256 rows, CUDA events around the selection inside the step): the split
-// path takes 98 us (its threshold, sweep and select kernels share it about 21 : 50 :
-// 29) against 78 us for one CTA per row. Each of the three is bound by fixed latency
+// path takes 85 us (three kernels) against 63 us for one CTA per row. Each of the
+// three is bound by fixed latency
 // (short-lived sweep CTAs in waves, and the block-wide radix passes of the threshold
 // and of the selection), so the forward keeps one CTA per row; the split path stays
 // available through dsa_topk_ws.

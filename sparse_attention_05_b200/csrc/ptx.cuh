@@ -228,6 +228,11 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, uint
       : "memory");
 }
 
+// Bulk prefetch of a contiguous global range into L2 (no completion to wait on):
+// src 16-B aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }

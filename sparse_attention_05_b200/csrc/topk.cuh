@@ -6,18 +6,22 @@
 // order-preserving 32-bit key (-0.0 maps to +0.0). The exact selection is a
 // radix select:
 //   find_kth   histograms of key bits [31:21], [20:10], [9:0] restricted to the
-//              prefix found so far -> the exact k-th largest key tau and the
-//              number r of keys equal to tau that belong to the selection;
+//              prefix found so far (one shared-memory atomic per key; grouping
+//              equal digits with match.any first measured slower) -> the exact
+//              k-th largest key tau and the number r of keys equal to tau that
+//              belong to the selection;
 //   compact    one ordered sweep: a key > tau is selected, a key == tau is
 //              selected while fewer than r equal keys precede it, so equal
 //              scores keep the lower position and the output is ascending.
 // Long rows (more than 4k keys) first shrink to a candidate list: a fixed
 // strided sample of 2048 scores gives a threshold that lies, with a wide
 // margin, below the k-th score; one coalesced sweep keeps the keys at or above
-// it in position order, and the exact selection runs on the candidates. The
-// candidates hold the k largest keys whenever there are at least k of them, so
-// the result is exact; if the sample misjudged (fewer than k candidates, or
-// more than the buffer holds) the row falls back to the exact full-row path.
+// it, and the exact selection runs on the candidates (rows of up to 131072 keys:
+// kept in any order and selected through bitmaps over the positions; longer
+// rows: kept in position order and compacted in order). The candidates hold the
+// k largest keys whenever there are at least k of them, so the result is exact;
+// if the sample misjudged (fewer than k candidates, or more than the buffer
+// holds) the row falls back to the exact full-row path.
 #pragma once
 
 #include "ptx.cuh"
@@ -31,7 +35,9 @@ constexpr int kTopkCandCap = kTopkCacheElems / 2;              // candidates: ke
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkBinsPerThread = 2048 / kTopkThreads;
 constexpr int kTopkSample = 2048;
-constexpr int kTopkSmemBytes = kTopkCacheElems * 4 + 2048 * 4 + 64 * 4 + kTopkSample * 4;
+// cache | hist | misc | sample, then the selection bitmaps of a long row (the second
+// one starts over the sample, which is dead by then): 4096 + 4096 words
+constexpr int kTopkSmemBytes = kTopkCacheElems * 4 + 2048 * 4 + 64 * 4 + 2 * 4096 * 4;
 
 struct TopkParams {
   const float* scores;
@@ -93,44 +99,76 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
 }
 
 // The k-th largest key among elements [0, n) (k <= n) and how many keys equal to
-// it belong to the top k. misc: [0..31] warp totals, [32] total, [33..34] result.
+// it belong to the top k. misc: [0..15] warp totals, [33..34] the pass's result.
+// Three barriers per pass: after the histogram, after the warps' bin totals, after
+// the result. Each thread owns four consecutive bins (walked from the top), reads
+// them once per pass and clears them for the next pass, so hist is all zero again
+// on return.
+// With passes = 2 only key bits [31:10] are resolved: tau is then the k-th largest
+// key with its low 10 bits cleared, a lower bound of it (r_eq is not meaningful).
 template <class KeyAt>
 __device__ void find_kth(int n, uint32_t k, KeyAt key_at, uint32_t* hist, uint32_t* misc,
-                         uint32_t& tau, uint32_t& r_eq) {
-  const int tid = threadIdx.x;
+                         uint32_t& tau, uint32_t& r_eq, int passes = 3) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n_iter = (n + kTopkThreads - 1) / kTopkThreads;
   uint32_t prefix = 0, prefix_mask = 0, remaining = k;
   const int shifts[3] = {21, 10, 0};
   const int widths[3] = {11, 11, 10};
+  for (int j = tid; j < 2048; j += kTopkThreads) hist[j] = 0;
+  __syncthreads();
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
+  for (int pass = 0; pass < passes; ++pass) {
     const int shift = shifts[pass];
     const uint32_t nbins = 1u << widths[pass];
-    for (int j = tid; j < 2048; j += kTopkThreads) hist[j] = 0;
-    __syncthreads();
+    // histogram of the digits of keys matching the prefix, four keys in flight
 #pragma unroll 1
-    for (int it = 0; it < n_iter; ++it) {
-      const int e = it * kTopkThreads + tid;
-      uint32_t digit = 0xFFFFFFFFu;
-      if (e < n) {
-        const uint32_t key = key_at(e, pass);
-        if ((key & prefix_mask) == prefix) digit = (key >> shift) & (nbins - 1);
+    for (int it = 0; it < n_iter; it += 4) {
+      uint32_t digit[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = (it + u) * kTopkThreads + tid;
+        digit[u] = 0xFFFFFFFFu;
+        if (e < n) {
+          const uint32_t key = key_at(e, pass);
+          if ((key & prefix_mask) == prefix) digit[u] = (key >> shift) & (nbins - 1);
+        }
       }
-      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-      if (digit != 0xFFFFFFFFu && (__ffs(peers) - 1) == (tid & 31))
-        atomicAdd(&hist[digit], __popc(peers));
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (digit[u] != 0xFFFFFFFFu) atomicAdd(&hist[digit[u]], 1u);
     }
     __syncthreads();
-    // the bin holding the remaining-th largest key: bins walked from the top,
-    // kTopkBinsPerThread consecutive ones per thread (2047 - B tid - i)
+    // the bin holding the remaining-th largest key: thread tid owns bins
+    // 2047 - B tid - i, i < B (B = kTopkBinsPerThread)
     uint32_t cnt[kTopkBinsPerThread], sum = 0;
 #pragma unroll
     for (int i = 0; i < kTopkBinsPerThread; ++i) {
       const int bin = 2047 - kTopkBinsPerThread * tid - i;
-      cnt[i] = bin < (int)nbins ? hist[bin] : 0u;
+      cnt[i] = 0u;
+      if (bin < (int)nbins) {
+        cnt[i] = hist[bin];
+        hist[bin] = 0u;
+      }
       sum += cnt[i];
     }
-    uint32_t above = block_exclusive_scan(sum, misc, misc + 32);
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) misc[warp] = incl;
+    __syncthreads();
+    uint32_t above = incl - sum;
+    {  // the totals of the warps before this one (four 16-B reads)
+      const uint4* t4 = reinterpret_cast<const uint4*>(misc);
+#pragma unroll
+      for (int q = 0; q < kTopkWarps / 4; ++q) {
+        const uint4 t = t4[q];
+        above += (4 * q + 0 < warp ? t.x : 0u) + (4 * q + 1 < warp ? t.y : 0u) +
+                 (4 * q + 2 < warp ? t.z : 0u) + (4 * q + 3 < warp ? t.w : 0u);
+      }
+    }
 #pragma unroll
     for (int i = 0; i < kTopkBinsPerThread; ++i) {
       if (above < remaining && remaining <= above + cnt[i]) {
@@ -144,7 +182,6 @@ __device__ void find_kth(int n, uint32_t k, KeyAt key_at, uint32_t* hist, uint32
     remaining = misc[34];
     prefix |= d << shift;
     prefix_mask |= (nbins - 1) << shift;
-    __syncthreads();
   }
   tau = prefix;
   r_eq = remaining;
@@ -233,14 +270,92 @@ __device__ void select_short_row(const float* row, int n, uint32_t k, float* cac
                  [&](int e) { return e; }, out, misc);
 }
 
+constexpr int kCandThreads = 512;
+static_assert(kCandThreads == kTopkThreads, "the shared selection code assumes one block shape");
+constexpr int kCandCap = 8192;                     // candidates per row staged in smem
+constexpr int kCandMaxWords = 4096;                // bitmap words: rows of <= 131072 keys
+
+// The exact top k of a row of n visible keys from m >= k candidates staged in
+// shared memory as (order-preserving key, position) in any order, when they hold
+// every key of the row at or above the row's k-th key: the k-th key tau and the
+// number r of equal keys to take (find_kth); every key at or above tau marked in a
+// bitmap over the row's positions; when more than r keys equal tau, the ones past
+// the r lowest positions (an ordered scan of a second bitmap of the equal keys)
+// unmarked again; the marks compacted in ascending order into out.
+// Bitmaps of (n + 31) / 32 <= kCandMaxWords words; misc[41] counts the equal keys.
+// Returns tau; with out == nullptr only tau is found.
+__device__ uint32_t select_from_candidates(int m, int n, uint32_t k, const uint32_t* ckey,
+                                           const int32_t* cpos, uint32_t* sel, uint32_t* tie,
+                                           uint32_t* hist, uint32_t* misc, int32_t* out) {
+  const int tid = threadIdx.x;
+  const int words = (n + 31) >> 5;
+  if (out) {  // ordered before their use by find_kth's first barrier
+    for (int w = tid; w < words; w += kTopkThreads) sel[w] = 0u;
+    if (tid == 0) misc[41] = 0u;
+  }
+  uint32_t tau, r_eq;
+  find_kth(m, k, [&](int e, int) { return ckey[e]; }, hist, misc, tau, r_eq);
+  if (!out) return tau;
+  for (int e = tid; e < m; e += kTopkThreads) {
+    const uint32_t key = ckey[e];
+    if (key >= tau) {
+      const int pos = cpos[e];
+      atomicOr(&sel[pos >> 5], 1u << (pos & 31));
+      if (key == tau) atomicAdd(&misc[41], 1u);
+    }
+  }
+  __syncthreads();
+  const int per = (words + kTopkThreads - 1) / kTopkThreads;
+  const int w0 = tid * per;
+  if (misc[41] > r_eq) {  // block-uniform: ties at tau reach past the selection
+    for (int w = tid; w < words; w += kTopkThreads) tie[w] = 0u;
+    __syncthreads();
+    for (int e = tid; e < m; e += kTopkThreads)
+      if (ckey[e] == tau) atomicOr(&tie[cpos[e] >> 5], 1u << (cpos[e] & 31));
+    __syncthreads();
+    // keep the r_eq lowest positions among the equal keys (each thread owns
+    // consecutive words of both bitmaps)
+    uint32_t cnt = 0;
+    for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(tie[w]);
+    uint32_t before = block_exclusive_scan(cnt, misc, misc + 32);
+    for (int w = w0; w < w0 + per && w < words; ++w) {
+      uint32_t bits = tie[w];
+      while (bits) {
+        const uint32_t bit = bits & (~bits + 1u);
+        if (before >= r_eq) sel[w] &= ~bit;
+        ++before;
+        bits ^= bit;
+      }
+    }
+    __syncthreads();
+  }
+  // ascending compaction of the selection (exactly k marks)
+  uint32_t cnt = 0;
+  for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(sel[w]);
+  uint32_t o = block_exclusive_scan(cnt, misc, misc + 32);
+  for (int w = w0; w < w0 + per && w < words; ++w) {
+    uint32_t bits = sel[w];
+    while (bits) {
+      const int bpos = __ffs(bits) - 1;
+      if (o < k) out[o] = w * 32 + bpos;
+      ++o;
+      bits &= bits - 1u;
+    }
+  }
+  return tau;
+}
+
 __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* cache = reinterpret_cast<float*>(smem_raw);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw + kTopkCacheElems * 4);
-  uint32_t* misc = hist + 2048;  // [0..31] warp totals, [32] total, [33..35] results
+  uint32_t* misc = hist + 2048;  // [0..31] warp totals, [32] total, [33..34] results,
+                                 // [41] equal keys, [48..63] per-warp kept-key counts
   uint32_t* sample = misc + 64;  // [kTopkSample]
   uint32_t* cand_key = reinterpret_cast<uint32_t*>(cache);      // [kTopkCandCap]
   int32_t* cand_pos = reinterpret_cast<int32_t*>(cache) + kTopkCandCap;
+  uint32_t* tie = sample;        // [kCandMaxWords] bitmaps of the long-row selection
+  uint32_t* sel = sample + kCandMaxWords;
 
   const int b = blockIdx.x / p.row_count;
   const int i = p.row_begin + blockIdx.x % p.row_count;
@@ -270,91 +385,218 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
 
   if (n > 4 * p.k) {
     // ---- candidate filter ------------------------------------------------------
-    // strided sample -> threshold with a wide safety margin below the k-th key
-    for (int s = tid; s < kTopkSample; s += kTopkThreads)
-      sample[s] = score_key(row[(int64_t)s * n / kTopkSample]);
+    // strided sample (a thread's four loads in flight) -> threshold with a wide
+    // safety margin below the k-th key
+    {
+      constexpr int kPer = kTopkSample / kTopkThreads;
+      uint32_t sk[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j)
+        sk[j] = score_key(row[(int64_t)(tid + j * kTopkThreads) * n / kTopkSample]);
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) sample[tid + j * kTopkThreads] = sk[j];
+    }
     __syncthreads();
     const float frac = (float)p.k / (float)n;
     const float expect = frac * kTopkSample;
     uint32_t r = (uint32_t)(expect + 4.0f * sqrtf(expect) + 16.0f);
     r = min(r, (uint32_t)kTopkSample);
+    // two radix passes: the r-th sample key with its low 10 bits cleared, which only
+    // lowers the threshold further
     uint32_t tau_low, unused;
-    find_kth(kTopkSample, r, [&](int e, int) { return sample[e]; }, hist, misc, tau_low, unused);
-    // keep keys >= tau_low in position order: 16 consecutive keys per thread
-    // per step, with the next step's four 16-B loads already in flight
-    constexpr int kStep = 16 * kTopkThreads;
-    auto load16 = [&](int base, float4 (&v)[4]) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e0 = base + 16 * tid + 4 * u;
-        if (e0 + 3 < n) {  // rows start 16-B aligned (ld is a multiple of 4)
-          v[u] = *reinterpret_cast<const float4*>(row + e0);
-        } else {
-          v[u].x = e0 < n ? row[e0] : -INFINITY;
-          v[u].y = e0 + 1 < n ? row[e0 + 1] : -INFINITY;
-          v[u].z = e0 + 2 < n ? row[e0 + 2] : -INFINITY;
-          v[u].w = e0 + 3 < n ? row[e0 + 3] : -INFINITY;
-        }
-      }
-    };
-    uint32_t m_run = 0;
-    bool overflow = false;
-    float4 cur4[4], nxt4[4];
-    load16(0, cur4);
+    find_kth(kTopkSample, r, [&](int e, int) { return sample[e]; }, hist, misc, tau_low, unused,
+             2);
     // key >= tau_low <=> score >= thr (order-preserving keys, -0.0 == +0.0, no NaN)
     const float thr = key_score(tau_low);
-#pragma unroll 1
-    for (int base = 0; base < n; base += kStep) {
-      if (base + kStep < n) load16(base + kStep, nxt4);
-      const int e0 = base + 16 * tid;
-      uint32_t mask = 0;  // bit u: key e0 + u is kept
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        mask |= (cur4[u].x >= thr ? 1u : 0u) << (4 * u);
-        mask |= (cur4[u].y >= thr ? 2u : 0u) << (4 * u);
-        mask |= (cur4[u].z >= thr ? 4u : 0u) << (4 * u);
-        mask |= (cur4[u].w >= thr ? 8u : 0u) << (4 * u);
-      }
-      if (base + kStep > n) {  // the last step: no key at or past n
-        const int left = n - e0;
-        mask &= left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u);
-      }
-      const uint32_t excl = block_exclusive_scan(__popc(mask), misc, misc + 32);
-      const uint32_t tot = misc[32];
-      uint32_t w = m_run + excl;
-      if (mask) {
-        auto put = [&](int u, float x) {
-          if ((mask >> u) & 1u) {
-            if (w < (uint32_t)kTopkCandCap) {
-              cand_key[w] = score_key(x);
-              cand_pos[w] = e0 + u;
-            }
-            ++w;
-          }
-        };
+    constexpr int kStep = 16 * kTopkThreads;
+
+    if (n <= kCandMaxWords * 32) {
+      // Unordered sweep: per step each warp reads 512 consecutive keys (four fully
+      // coalesced 16-B loads per lane, the next step's in flight) and appends the
+      // positions of its kept keys to a region of its own (a warp scan places them;
+      // each lane stores one position per kept key), so no step waits on a block
+      // barrier or a shared counter. Afterwards the regions are packed and the kept
+      // keys re-read from the row (in L2 by then). The selection from the candidates
+      // works through bitmaps over the row's positions, so their order does not
+      // matter. Every warp sees 512 of each 8192 keys, so the regions fill evenly.
+      constexpr int kWarpCap = kTopkCandCap / kTopkWarps;  // 512 positions per warp
+      const int lane = tid & 31, warp = tid >> 5, wbase = warp * 512 + 4 * lane;
+      int32_t* wpos = cand_pos + warp * kWarpCap;
+      auto load16 = [&](int base, float4 (&v)[4]) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          put(4 * u, cur4[u].x);
-          put(4 * u + 1, cur4[u].y);
-          put(4 * u + 2, cur4[u].z);
-          put(4 * u + 3, cur4[u].w);
+          const int e0 = base + wbase + 128 * u;
+          if (e0 + 3 < n) {  // rows start 16-B aligned (ld is a multiple of 4)
+            v[u] = *reinterpret_cast<const float4*>(row + e0);
+          } else {
+            v[u].x = e0 < n ? row[e0] : -INFINITY;
+            v[u].y = e0 + 1 < n ? row[e0 + 1] : -INFINITY;
+            v[u].z = e0 + 2 < n ? row[e0 + 2] : -INFINITY;
+            v[u].w = e0 + 3 < n ? row[e0 + 3] : -INFINITY;
+          }
         }
-      }
-      m_run += tot;
-      overflow = m_run > (uint32_t)kTopkCandCap;
-      __syncthreads();
-      if (overflow) break;
+      };
+      // The row streams into L2 a few steps ahead of the loads (one thread issues
+      // bulk prefetches).
+      constexpr int kAhead = 3;
+      auto prefetch_step = [&](int start) {
+        if (tid == 0 && start < n) {
+          const int cnt = min(kStep, n - start) & ~3;  // whole 16-B pieces
+          if (cnt > 0) prefetch_l2_bulk(row + start, (uint32_t)cnt * 4u);
+        }
+      };
 #pragma unroll
-      for (int u = 0; u < 4; ++u) cur4[u] = nxt4[u];
-    }
-    if (!overflow && m_run >= k) {
-      const int m = (int)m_run;
-      find_kth(m, k, [&](int e, int) { return cand_key[e]; }, hist, misc, tau, r_eq);
-      if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = key_score(tau);
-      if (out)
-        compact_topk(m, tau, r_eq, [&](int e, int) { return cand_key[e]; },
-                     [&](int e) { return cand_pos[e]; }, out, misc);
-      return;
+      for (int j = 1; j <= kAhead; ++j) prefetch_step(j * kStep);
+      uint32_t wcount = 0;  // warp-uniform: kept keys this warp has found
+      float4 cur4[4], nxt4[4];
+      load16(0, cur4);
+#pragma unroll 1
+      for (int base = 0; base < n; base += kStep) {
+        prefetch_step(base + (kAhead + 1) * kStep);
+        if (base + kStep < n) load16(base + kStep, nxt4);
+        uint32_t mask = 0;  // bit 4u + j: key base + wbase + 128u + j is kept
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e0 = base + wbase + 128 * u;
+          uint32_t m4 = (cur4[u].x >= thr ? 1u : 0u) | (cur4[u].y >= thr ? 2u : 0u) |
+                        (cur4[u].z >= thr ? 4u : 0u) | (cur4[u].w >= thr ? 8u : 0u);
+          if (base + kStep > n) {  // the last step: no key at or past n
+            const int left = n - e0;
+            m4 &= left >= 4 ? 0xFu : (left <= 0 ? 0u : (1u << left) - 1u);
+          }
+          mask |= m4 << (4 * u);
+        }
+        const uint32_t c = __popc(mask);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        uint32_t w = wcount + incl - c;
+        while (mask) {
+          const int bit = __ffs(mask) - 1;
+          if (w < (uint32_t)kWarpCap) wpos[w] = base + wbase + 128 * (bit >> 2) + (bit & 3);
+          ++w;
+          mask &= mask - 1u;
+        }
+        wcount += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) cur4[u] = nxt4[u];
+      }
+      if (lane == 0) misc[48 + warp] = wcount;
+      __syncthreads();
+      uint32_t m = 0, off = 0;
+      bool fits = true;
+#pragma unroll
+      for (int v = 0; v < kTopkWarps; ++v) {
+        const uint32_t cv = misc[48 + v];
+        fits = fits && cv <= (uint32_t)kWarpCap;
+        off += v < warp ? cv : 0u;
+        m += cv;
+      }
+      if (fits && m >= k) {
+        // pack the regions (positions held in registers across the barrier) and
+        // fetch the keys of the kept positions
+        constexpr int kPer = kWarpCap / 32;
+        int32_t pos[kPer];
+        float x[kPer];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const uint32_t e = (uint32_t)(lane + 32 * j);
+          pos[j] = e < wcount ? wpos[e] : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) x[j] = row[pos[j]];
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const uint32_t e = (uint32_t)(lane + 32 * j);
+          if (e < wcount) {
+            cand_pos[off + e] = pos[j];
+            cand_key[off + e] = score_key(x[j]);
+          }
+        }
+        __syncthreads();  // the packed list, and misc, before the selection
+        const uint32_t tau_c =
+            select_from_candidates((int)m, n, k, cand_key, cand_pos, sel, tie, hist, misc, out);
+        if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = key_score(tau_c);
+        return;
+      }
+    } else {
+      // Rows longer than the bitmaps: keep keys >= tau_low in position order, 16
+      // consecutive keys per thread per step (a block scan places them).
+      auto load16 = [&](int base, float4 (&v)[4]) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e0 = base + 16 * tid + 4 * u;
+          if (e0 + 3 < n) {
+            v[u] = *reinterpret_cast<const float4*>(row + e0);
+          } else {
+            v[u].x = e0 < n ? row[e0] : -INFINITY;
+            v[u].y = e0 + 1 < n ? row[e0 + 1] : -INFINITY;
+            v[u].z = e0 + 2 < n ? row[e0 + 2] : -INFINITY;
+            v[u].w = e0 + 3 < n ? row[e0 + 3] : -INFINITY;
+          }
+        }
+      };
+      uint32_t m_run = 0;
+      bool overflow = false;
+      float4 cur4[4], nxt4[4];
+      load16(0, cur4);
+#pragma unroll 1
+      for (int base = 0; base < n; base += kStep) {
+        if (base + kStep < n) load16(base + kStep, nxt4);
+        const int e0 = base + 16 * tid;
+        uint32_t mask = 0;  // bit u: key e0 + u is kept
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          mask |= (cur4[u].x >= thr ? 1u : 0u) << (4 * u);
+          mask |= (cur4[u].y >= thr ? 2u : 0u) << (4 * u);
+          mask |= (cur4[u].z >= thr ? 4u : 0u) << (4 * u);
+          mask |= (cur4[u].w >= thr ? 8u : 0u) << (4 * u);
+        }
+        if (base + kStep > n) {  // the last step: no key at or past n
+          const int left = n - e0;
+          mask &= left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u);
+        }
+        const uint32_t excl = block_exclusive_scan(__popc(mask), misc, misc + 32);
+        const uint32_t tot = misc[32];
+        uint32_t w = m_run + excl;
+        if (mask) {
+          auto put = [&](int u, float x) {
+            if ((mask >> u) & 1u) {
+              if (w < (uint32_t)kTopkCandCap) {
+                cand_key[w] = score_key(x);
+                cand_pos[w] = e0 + u;
+              }
+              ++w;
+            }
+          };
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            put(4 * u, cur4[u].x);
+            put(4 * u + 1, cur4[u].y);
+            put(4 * u + 2, cur4[u].z);
+            put(4 * u + 3, cur4[u].w);
+          }
+        }
+        m_run += tot;
+        overflow = m_run > (uint32_t)kTopkCandCap;
+        __syncthreads();
+        if (overflow) break;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) cur4[u] = nxt4[u];
+      }
+      if (!overflow && m_run >= k) {
+        const int m = (int)m_run;
+        find_kth(m, k, [&](int e, int) { return cand_key[e]; }, hist, misc, tau, r_eq);
+        if (p.kth_out && tid == 0) p.kth_out[blockIdx.x] = key_score(tau);
+        if (out)
+          compact_topk(m, tau, r_eq, [&](int e, int) { return cand_key[e]; },
+                       [&](int e) { return cand_pos[e]; }, out, misc);
+        return;
+      }
     }
     // the sample misjudged this row: exact selection over the whole row
     __syncthreads();
@@ -381,11 +623,6 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
 // above tau marked in a bitmap over the row's positions, the r lowest positions of
 // the keys equal to tau marked from a second bitmap, and the marks compacted in
 // ascending order. Other rows are listed for the full (unfused) selection.
-constexpr int kCandThreads = 512;
-static_assert(kCandThreads == kTopkThreads, "the shared selection code assumes one block shape");
-constexpr int kCandCap = 8192;                     // candidates per row staged in smem
-constexpr int kCandMaxWords = 4096;                // bitmap words: rows of <= 131072 keys
-
 struct CandParams {
   const uint32_t* cand_key;  // [batch * row_count][cand_cap]
   const int32_t* cand_pos;   // [batch * row_count][cand_cap]
@@ -402,61 +639,6 @@ struct CandParams {
 
 constexpr int kCandSmemBytes =
     kCandCap * 8 + 2 * kCandMaxWords * 4 + 2048 * 4 + 64 * 4;
-
-// The exact top k of a row of n visible keys from m >= k candidates staged in
-// shared memory as (order-preserving key, position) in any order, when they hold
-// every key of the row at or above the row's k-th key: the k-th key tau and the
-// number r of equal keys to take (find_kth), keys above tau marked in a bitmap over
-// the row's positions, the r lowest positions among the keys equal to tau marked
-// from a second bitmap, and the marks compacted in ascending order into out.
-// Bitmaps of (n + 31) / 32 <= kCandMaxWords words.
-__device__ void select_from_candidates(int m, int n, uint32_t k, const uint32_t* ckey,
-                                       const int32_t* cpos, uint32_t* sel, uint32_t* tie,
-                                       uint32_t* hist, uint32_t* misc, int32_t* out) {
-  const int tid = threadIdx.x;
-  const int words = (n + 31) >> 5;
-  for (int w = tid; w < words; w += kTopkThreads) sel[w] = tie[w] = 0u;
-  __syncthreads();
-  uint32_t tau, r_eq;
-  find_kth(m, k, [&](int e, int) { return ckey[e]; }, hist, misc, tau, r_eq);
-  for (int e = tid; e < m; e += kTopkThreads) {
-    const uint32_t key = ckey[e];
-    const int pos = cpos[e];
-    if (key > tau) atomicOr(&sel[pos >> 5], 1u << (pos & 31));
-    else if (key == tau) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
-  }
-  __syncthreads();
-  // the r_eq lowest positions among the keys equal to tau: an ordered scan of the
-  // tie bitmap (each thread owns consecutive words)
-  const int per = (words + kTopkThreads - 1) / kTopkThreads;
-  const int w0 = tid * per;
-  uint32_t cnt = 0;
-  for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(tie[w]);
-  uint32_t before = block_exclusive_scan(cnt, misc, misc + 32);
-  for (int w = w0; w < w0 + per && w < words; ++w) {
-    uint32_t bits = tie[w];
-    while (bits) {
-      const uint32_t bit = bits & (~bits + 1u);
-      if (before < r_eq) sel[w] |= bit;
-      ++before;
-      bits ^= bit;
-    }
-  }
-  __syncthreads();
-  // ascending compaction of the selection (exactly k marks)
-  cnt = 0;
-  for (int w = w0; w < w0 + per && w < words; ++w) cnt += __popc(sel[w]);
-  uint32_t o = block_exclusive_scan(cnt, misc, misc + 32);
-  for (int w = w0; w < w0 + per && w < words; ++w) {
-    uint32_t bits = sel[w];
-    while (bits) {
-      const int bpos = __ffs(bits) - 1;
-      if (o < k) out[o] = w * 32 + bpos;
-      ++o;
-      bits &= bits - 1u;
-    }
-  }
-}
 
 __global__ void __launch_bounds__(kCandThreads, 2) cand_select_kernel(CandParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -545,12 +727,12 @@ __device__ __forceinline__ int split_row(const SplitParams& p, int64_t wrow, int
   return R.seqlen - R.q_len + i + 1;
 }
 
-// Threshold key of a long row, the one topk_kernel's one-CTA path uses: the r-th
-// largest of the fixed strided sample of 2048 scores, r = the expected count of top-k
-// keys in the sample + 4 standard deviations + 16. One CTA of 4 warps per row computes
-// it: each thread holds 16 sampled keys, and four passes over 8-bit digits (a
-// 256-bin histogram with match.any-aggregated shared atomics, then a scan of the bins
-// by warp 0) narrow the prefix down to the exact key.
+// Threshold key of a long row: the r-th largest of the fixed strided sample of 2048
+// scores, r = the expected count of top-k keys in the sample + 4 standard deviations
+// + 16 (topk_kernel's one-CTA path takes the same key with its low 10 bits cleared).
+// One CTA of 4 warps per row computes it: each thread holds 16 sampled keys, and four
+// passes over 8-bit digits (a 256-bin histogram of shared atomics, then a scan of the
+// bins by warp 0) narrow the prefix down to the exact key.
 constexpr int kThresholdThreads = 128;
 
 __device__ __forceinline__ uint32_t sample_threshold(const float* row, int n, uint32_t k,
@@ -572,8 +754,7 @@ __device__ __forceinline__ uint32_t sample_threshold(const float* row, int n, ui
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const uint32_t digit = (key[j] & mask) == prefix ? (key[j] >> shift) & 255u : 256u;
-      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-      if (digit < 256u && (__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], __popc(peers));
+      if (digit < 256u) atomicAdd(&hist[digit], 1u);
     }
     __syncthreads();
     if (warp == 0) {  // bins from the top: lane l owns bins 255 - 8 l - i, i < 8
