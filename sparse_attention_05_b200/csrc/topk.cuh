@@ -112,14 +112,12 @@ __device__ void find_kth(int n, uint32_t k, KeyAt key_at, uint32_t* hist, uint32
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n_iter = (n + kTopkThreads - 1) / kTopkThreads;
   uint32_t prefix = 0, prefix_mask = 0, remaining = k;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
   for (int j = tid; j < 2048; j += kTopkThreads) hist[j] = 0;
   __syncthreads();
 #pragma unroll 1
   for (int pass = 0; pass < passes; ++pass) {
-    const int shift = shifts[pass];
-    const uint32_t nbins = 1u << widths[pass];
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);  // key bits [31:21] [20:10] [9:0]
+    const uint32_t nbins = pass == 2 ? 1024u : 2048u;
     // histogram of the digits of keys matching the prefix, four keys in flight
 #pragma unroll 1
     for (int it = 0; it < n_iter; it += 4) {
@@ -412,33 +410,35 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
 
     if (n <= kCandMaxWords * 32) {
       // Unordered sweep: per step each warp reads 512 consecutive keys (four fully
-      // coalesced 16-B loads per lane, the next step's in flight) and appends the
-      // positions of its kept keys to a region of its own (a warp scan places them;
-      // each lane stores one position per kept key), so no step waits on a block
-      // barrier or a shared counter. Afterwards the regions are packed and the kept
-      // keys re-read from the row (in L2 by then). The selection from the candidates
-      // works through bitmaps over the row's positions, so their order does not
-      // matter. Every warp sees 512 of each 8192 keys, so the regions fill evenly.
+      // coalesced 16-B pieces per lane) and appends the positions of its kept keys to
+      // a region of its own (a warp scan places them; each lane stores one position
+      // per kept key), so no step waits on a block barrier or a shared counter. Each
+      // lane's pieces arrive by cp.async two steps ahead in one of two 32 KB slots
+      // (the candidate keys' and the bitmaps' space, both free until the sweep ends),
+      // and each lane reads back only its own pieces, so its cp.async waits are the
+      // only synchronisation. Afterwards the regions are packed and the kept keys
+      // re-read from the row (in L2 by then). The selection from the candidates works
+      // through bitmaps over the row's positions, so their order does not matter.
+      // Every warp sees 512 of each 8192 keys, so the regions fill evenly.
       constexpr int kWarpCap = kTopkCandCap / kTopkWarps;  // 512 positions per warp
       const int lane = tid & 31, warp = tid >> 5, wbase = warp * 512 + 4 * lane;
       int32_t* wpos = cand_pos + warp * kWarpCap;
-      auto load16 = [&](int base, float4 (&v)[4]) {
+      const uint32_t slot0 = smem_u32(cache), slot1 = smem_u32(tie);
+      // this lane's four pieces of the step at `base` into slot `sl` (zero fill past n;
+      // those keys are masked)
+      auto copy_step = [&](int base, int sl) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int e0 = base + wbase + 128 * u;
-          if (e0 + 3 < n) {  // rows start 16-B aligned (ld is a multiple of 4)
-            v[u] = *reinterpret_cast<const float4*>(row + e0);
-          } else {
-            v[u].x = e0 < n ? row[e0] : -INFINITY;
-            v[u].y = e0 + 1 < n ? row[e0 + 1] : -INFINITY;
-            v[u].z = e0 + 2 < n ? row[e0 + 2] : -INFINITY;
-            v[u].w = e0 + 3 < n ? row[e0 + 3] : -INFINITY;
-          }
+          const int left = n - e0;
+          const uint32_t bytes = left >= 4 ? 16u : (left <= 0 ? 0u : 4u * (uint32_t)left);
+          cp_async_16((sl ? slot1 : slot0) + (uint32_t)(wbase + 128 * u) * 4u,
+                      bytes ? row + e0 : row, bytes);
         }
+        cp_async_commit();
       };
-      // The row streams into L2 a few steps ahead of the loads (one thread issues
-      // bulk prefetches).
-      constexpr int kAhead = 3;
+      // The row also streams into L2 a few steps ahead (one thread's bulk prefetches).
+      constexpr int kAhead = 4;
       auto prefetch_step = [&](int start) {
         if (tid == 0 && start < n) {
           const int cnt = min(kStep, n - start) & ~3;  // whole 16-B pieces
@@ -446,14 +446,21 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
         }
       };
 #pragma unroll
-      for (int j = 1; j <= kAhead; ++j) prefetch_step(j * kStep);
+      for (int j = 2; j <= kAhead; ++j) prefetch_step(j * kStep);
+      copy_step(0, 0);
+      if (kStep < n) copy_step(kStep, 1);
       uint32_t wcount = 0;  // warp-uniform: kept keys this warp has found
-      float4 cur4[4], nxt4[4];
-      load16(0, cur4);
 #pragma unroll 1
-      for (int base = 0; base < n; base += kStep) {
+      for (int base = 0, sl = 0; base < n; base += kStep, sl ^= 1) {
         prefetch_step(base + (kAhead + 1) * kStep);
-        if (base + kStep < n) load16(base + kStep, nxt4);
+        if (base + kStep < n) cp_async_wait_group<1>();  // this step's pieces have landed
+        else cp_async_wait_group<0>();
+        float4 cur4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float* src = (sl == 0 ? cache : reinterpret_cast<const float*>(tie)) + wbase + 128 * u;
+          cur4[u] = *reinterpret_cast<const float4*>(src);
+        }
         uint32_t mask = 0;  // bit 4u + j: key base + wbase + 128u + j is kept
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -466,6 +473,9 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
           }
           mask |= m4 << (4 * u);
         }
+        // the slot is free again once its values are in registers (the mask above
+        // depends on all four reads): the step two ahead goes into it
+        if (base + 2 * kStep < n) copy_step(base + 2 * kStep, sl);
         const uint32_t c = __popc(mask);
         uint32_t incl = c;
 #pragma unroll
@@ -481,9 +491,8 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
           mask &= mask - 1u;
         }
         wcount += __shfl_sync(0xffffffffu, incl, 31);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) cur4[u] = nxt4[u];
       }
+      cp_async_wait_all();
       if (lane == 0) misc[48 + warp] = wcount;
       __syncthreads();
       uint32_t m = 0, off = 0;
