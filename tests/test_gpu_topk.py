@@ -128,3 +128,19 @@ def test_split_chunk_edges_and_hot_ties():
     s[:, 16380:16390] = 9.0  # ties straddling the first chunk edge
     got, want = _run(s, seqlens, 1, 2048)
     np.testing.assert_array_equal(got, want)
+
+
+def test_rows_longer_than_the_position_bitmaps():
+    """Rows of more than 131072 keys keep their candidates in position order (the
+    bitmap selection covers shorter rows only): plain, tie-heavy and sample-misjudged
+    rows must still match the oracle exactly."""
+    rng = np.random.default_rng(13)
+    ld = 200000
+    seqlens = [200000, 150001, 131073, 199999]
+    s = rng.standard_normal((4, ld)).astype(np.float32)
+    pool = np.array([0.0, -0.0, 1.0, 1.5, 2.0, -3.0, 7.25], np.float32)
+    s[1] = rng.choice(pool, size=ld)
+    sampled = (np.arange(2048, dtype=np.int64) * seqlens[3]) // 2048
+    s[3][sampled] = 100.0 + rng.random(2048).astype(np.float32)  # threshold too high
+    got, want = _run(s, seqlens, 1, 2048)
+    np.testing.assert_array_equal(got, want)
