@@ -29,7 +29,8 @@
 //               can run that many tiles ahead; thread = key lane, which loads
 //               its key's scale from global memory itself, one tile ahead
 // A stage of the ring carries key codes only and is reused as soon as the MMA has
-// read it (the scales never gate a stage).
+// read it (the scales never gate a stage); the same commit tells the epilogue that
+// the tile's accumulator is ready.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -236,9 +237,13 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
   float* wq = reinterpret_cast<float*>(qbuf + 2 * kIdxQBufBytes);  // [2][256]
   uint64_t* bars = reinterpret_cast<uint64_t*>(wq + 2 * 4 * kIdxHeads);
   uint64_t* kfull = bars;
+  // kempty[s]: the MMAs of the tile in stage s are done, so its key stage is free and
+  // its accumulator holds the scores (one commit per tile serves the producer and the
+  // epilogue; the epilogue of a tile always observes that phase before the next tile
+  // in the same stage can finish, because that tile needs the accumulator this
+  // epilogue or a later one of the same warpgroup frees)
   uint64_t* kempty = bars + kIdxStages;
-  uint64_t* tfull = bars + 2 * kIdxStages;
-  uint64_t* tempty = tfull + kIdxMaxAcc;
+  uint64_t* tempty = bars + 2 * kIdxStages + kIdxMaxAcc;
   uint64_t* qfull = tempty + kIdxMaxAcc;
   uint64_t* qempty = qfull + 2;
   uint64_t* mdone = qempty + 2;
@@ -261,12 +266,9 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
     for (int s = 0; s < kIdxStages; ++s) {
       // expect_tx arrival (+ the TMA bytes), and one arrival per copy thread
       mbar_init(smem_u32(&kfull[s]), kAssist ? 1 + kIdxCpThreads : 1);
-      mbar_init(smem_u32(&kempty[s]), 1);  // the MMA's commit
+      mbar_init(smem_u32(&kempty[s]), 1);  // the MMA's commit (stage free, scores ready)
     }
-    for (int i = 0; i < kIdxMaxAcc; ++i) {
-      mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), 128);
-    }
+    for (int i = 0; i < kIdxMaxAcc; ++i) mbar_init(smem_u32(&tempty[i]), 128);
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&qfull[i]), 64);
       mbar_init(smem_u32(&qempty[i]), 1 + 256);
@@ -381,7 +383,6 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
             mma_fp8_ss(dcol, adesc, bdesc, idesc, kk > 0);
           }
           mma_commit(smem_u32(&kempty[st]));
-          mma_commit(smem_u32(&tfull[ab]));
         }
         if (!ok) break;
         mma_commit(smem_u32(&qempty[qb]));
@@ -570,7 +571,7 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
           pf_kt = kt + 2;
         }
         const int ab = (int)(it % (uint32_t)nacc);  // accumulator of this tile
-        if (!warp_wait(smem_u32(&tfull[ab]), (it / nacc) & 1, TO, abort_flag)) {
+        if (!warp_wait(smem_u32(&kempty[it % kIdxStages]), (it / kIdxStages) & 1, TO, abort_flag)) {
           ok = false;
           break;
         }
