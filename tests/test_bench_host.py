@@ -43,6 +43,38 @@ def test_job_throughput():
     assert bench.job_throughput(4, 256, 10, 2.0) == 4 * 256 * 10 / 2.0
 
 
+def test_step_roofline_sums_every_kernel():
+    peaks = {"hbm_gbs": 5000.0, "bf16_tflops": 1000.0, "bf16_tflops_sustained": 800.0}
+    work = {"a": {"bytes": 5e9, "flop": 0, "flop_dtype": None},          # 1 ms of HBM
+            "b": {"bytes": 5e9, "flop": 2e12, "flop_dtype": "bf16"},     # 1 ms, 2 ms of BF16
+            "c": {"bytes": 0, "flop": 4e12, "flop_dtype": "fp8"}}        # 2 ms of FP8
+    r = bench.step_roofline(work, ("a", "b", "c"), 8e-3, peaks, long_step=False)
+    assert abs(r["hbm_ms"] - 2.0) < 1e-9 and abs(r["tensor_ms"] - 4.0) < 1e-9
+    assert r["bound"] == "tensor" and abs(r["frac"] - 0.5) < 1e-12
+    r = bench.step_roofline(work, ("a", "b"), 4e-3, peaks, long_step=True)
+    assert abs(r["tensor_ms"] - 2.5) < 1e-9 and r["bound"] == "tensor"
+
+
+def test_end_to_end_staging_layout():
+    """The end-to-end run packs a step's inputs (and its outputs) into one buffer:
+    every tensor sits at a 256-byte boundary, views round-trip the data, and the
+    packed size is what one copy moves."""
+    t = {"q": torch.randn(3, 5).to(torch.bfloat16), "seqlens": torch.arange(7, dtype=torch.int32),
+         "w": torch.rand(2, 3), "table": torch.arange(12, dtype=torch.int32).view(3, 4)}
+    offs, total = bench._packed(t)
+    assert all(o % 256 == 0 for o in offs.values())
+    sizes = {n: v.numel() * v.element_size() for n, v in t.items()}
+    spans = sorted((offs[n], offs[n] + sizes[n]) for n in t)
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))  # no overlap
+    assert total >= spans[-1][1] and total % 256 == 0
+    blob = torch.zeros(total, dtype=torch.uint8)
+    for n, v in bench._views(blob, t, offs).items():
+        assert v.is_contiguous() and v.dtype == t[n].dtype and v.shape == t[n].shape
+        v.copy_(t[n])
+    back = bench._views(blob, t, offs)
+    assert all(torch.equal(back[n], t[n]) for n in t)
+
+
 def _worker(rank, world, port, results):
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
                             world_size=world)
