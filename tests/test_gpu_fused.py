@@ -78,6 +78,20 @@ def test_against_the_oracle():
     check_index_sets(got, topk_rows(sc, a["q_pos"], 2048), sc, a["q_pos"], 2048)
 
 
+def test_paged_long_rows_against_the_oracle():
+    """Paged varlen decode with rows past 4k keys (the sampled threshold and the
+    filtering pass decide them): the fused selection against the oracle's top-k of
+    the oracle's scores."""
+    p = synth.paged_decode(batch=3, q_per_seq=2, min_ctx=9000, max_ctx=20000, page_size=64,
+                           seed=129)
+    got, _ = _both(p)
+    a = oracle_args(p)
+    sc = indexer_scores(a["q_idx"], a["w"], a["k_idx"], a["k_scale"], a["q_seq"], a["q_pos"],
+                        ld=(p.max_ctx + 127) // 128 * 128,
+                        block_table=a["block_table"], page_size=p.page_size)
+    check_index_sets(got, topk_rows(sc, a["q_pos"], 2048), sc, a["q_pos"], 2048)
+
+
 def test_fused_forward_equals_forward():
     dsa = _dsa()
     p = synth.paged_decode(batch=4, q_per_seq=2, min_ctx=3000, max_ctx=16000, page_size=64,
