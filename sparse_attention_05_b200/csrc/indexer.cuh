@@ -57,6 +57,14 @@ constexpr int kIdxSmemBytes =
     2 * 4 * kIdxHeads * 4 /*wq*/ + 512 /*barriers etc*/ + 512 /*share + scan scratch*/ +
     2 * 4 * 256 * 4 /*filter mode: candidate keys staged for one tile*/;
 constexpr int kIdxMaxAcc = 8;  // TMEM accumulators: 512 / N, at most 8
+// Lean decode form (groups of at most two rows): two CTAs per SM, each with seven warps
+// (producer, MMA, one quantizer, one epilogue warpgroup), four key stages and half of
+// the SM's tensor memory, so that two independent tile pipelines share each SM.
+constexpr int kIdxLeanThreads = 224;
+constexpr int kIdxLeanStages = 4;
+constexpr int kIdxLeanQBufBytes = 2 * kIdxHeads * kIdxDim;  // G <= 2 rows x 64 heads x 128 B
+constexpr int kIdxLeanSmemBytes = 1024 + kIdxLeanStages * kIdxStageBytes +
+                                  2 * kIdxLeanQBufBytes + 2 * 4 * kIdxHeads * 4 + 512 + 512;
 
 struct IndexerParams {
   const __nv_bfloat16* q_idx;  // [T][64][128]
@@ -224,17 +232,21 @@ __device__ void idx_share(const IndexerParams& p, IdxShare* out, uint32_t* scrat
 // so the tile stream was bound by the TMA unit; the copy warps take half of it. The
 // 16 warps leave 128 registers per thread, so the epilogue reads tensor memory in
 // 16-column chunks.
-template <bool kFilter, bool kAssist = false>
-__global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
+template <bool kFilter, bool kAssist = false, bool kLean = false>
+__global__ void __launch_bounds__(kLean ? kIdxLeanThreads : (kAssist ? kIdxAssistThreads : kIdxThreads),
+                                  kLean ? 2 : 1)
     indexer_kernel(const __grid_constant__ IndexerParams p,
                    const __grid_constant__ CUtensorMap tm_keys) {
   static_assert(!(kFilter && kAssist), "the copy-assisted form is for plain scores");
+  static_assert(!(kLean && (kFilter || kAssist)), "the lean form is for plain scores");
+  constexpr int kS = kLean ? kIdxLeanStages : kIdxStages;        // key stages
+  constexpr int kQB = kLean ? kIdxLeanQBufBytes : kIdxQBufBytes;  // one query buffer
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* qbuf = stages + kIdxStages * kIdxStageBytes;
-  float* wq = reinterpret_cast<float*>(qbuf + 2 * kIdxQBufBytes);  // [2][256]
+  uint8_t* qbuf = stages + kS * kIdxStageBytes;
+  float* wq = reinterpret_cast<float*>(qbuf + 2 * kQB);  // [2][256]
   uint64_t* bars = reinterpret_cast<uint64_t*>(wq + 2 * 4 * kIdxHeads);
   uint64_t* kfull = bars;
   // kempty[s]: the MMAs of the tile in stage s are done, so its key stage is free and
@@ -242,8 +254,8 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
   // epilogue; the epilogue of a tile always observes that phase before the next tile
   // in the same stage can finish, because that tile needs the accumulator this
   // epilogue or a later one of the same warpgroup frees)
-  uint64_t* kempty = bars + kIdxStages;
-  uint64_t* tempty = bars + 2 * kIdxStages + kIdxMaxAcc;
+  uint64_t* kempty = bars + kS;
+  uint64_t* tempty = bars + 2 * kS + kIdxMaxAcc;
   uint64_t* qfull = tempty + kIdxMaxAcc;
   uint64_t* qempty = qfull + 2;
   uint64_t* mdone = qempty + 2;
@@ -259,19 +271,19 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
   // As many accumulators as tensor memory holds (an even number, so a given
   // accumulator always belongs to the same epilogue warpgroup): the MMA runs
   // up to nacc tiles ahead of the epilogue.
-  const int nacc = min(kIdxMaxAcc, 512 / N) & ~1;
-  const uint32_t tmem_cols = 512;
+  const uint32_t tmem_cols = kLean ? 256 : 512;
+  const int nacc = min(kIdxMaxAcc, (int)tmem_cols / N) & ~1;
 
   if (tid == 0) {
-    for (int s = 0; s < kIdxStages; ++s) {
+    for (int s = 0; s < kS; ++s) {
       // expect_tx arrival (+ the TMA bytes), and one arrival per copy thread
       mbar_init(smem_u32(&kfull[s]), kAssist ? 1 + kIdxCpThreads : 1);
       mbar_init(smem_u32(&kempty[s]), 1);  // the MMA's commit (stage free, scores ready)
     }
     for (int i = 0; i < kIdxMaxAcc; ++i) mbar_init(smem_u32(&tempty[i]), 128);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&qfull[i]), 64);
-      mbar_init(smem_u32(&qempty[i]), 1 + 256);
+      mbar_init(smem_u32(&qfull[i]), kLean ? 32 : 64);  // the quantizer warps' lanes
+      mbar_init(smem_u32(&qempty[i]), 1 + (kLean ? 128 : 256));  // MMA commit + epilogue
     }
     mbar_init(smem_u32(mdone), 1);
     *abort_flag = 0;
@@ -316,8 +328,8 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
           pg_cur = pg_nxt;
           pg_nxt = fetch_pages(kb + 16);
         }
-        const int st = it % kIdxStages;
-        if (!warp_wait(smem_u32(&kempty[st]), ((it / kIdxStages) & 1) ^ 1, TO, abort_flag)) {
+        const int st = it % kS;
+        if (!warp_wait(smem_u32(&kempty[st]), ((it / kS) & 1) ^ 1, TO, abort_flag)) {
           ok = false;
           break;
         }
@@ -350,8 +362,8 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
     }
     // Drain: the last stages' copies must land before the CTA may exit.
     if (lane == 0)
-      for (uint32_t j = it > kIdxStages ? it - kIdxStages : 0; j < it; ++j)
-        mbar_wait(smem_u32(&kfull[j % kIdxStages]), (j / kIdxStages) & 1, TO, no_abort);
+      for (uint32_t j = it > kS ? it - kS : 0; j < it; ++j)
+        mbar_wait(smem_u32(&kfull[j % kS]), (j / kS) & 1, TO, no_abort);
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -363,11 +375,11 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
       while (!*abort_flag && idx_next(p, sh, cur, U)) {
         const int qb = un & 1;
         if (!mbar_wait(smem_u32(&qfull[qb]), (un >> 1) & 1, TO, abort_flag)) break;
-        const uint32_t qaddr = smem_u32(qbuf + qb * kIdxQBufBytes);
+        const uint32_t qaddr = smem_u32(qbuf + qb * kQB);
         bool ok = true;
         for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
-          const int st = it % kIdxStages, ab = it % nacc;
-          if (!mbar_wait(smem_u32(&kfull[st]), (it / kIdxStages) & 1, TO, abort_flag) ||
+          const int st = it % kS, ab = it % nacc;
+          if (!mbar_wait(smem_u32(&kfull[st]), (it / kS) & 1, TO, abort_flag) ||
               !mbar_wait(smem_u32(&tempty[ab]), ((it / nacc) & 1) ^ 1, TO, abort_flag)) {
             ok = false;
             break;
@@ -407,8 +419,8 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
     while (ok && !*abort_flag && idx_next(p, sh, cur, U)) {
       const int pos_max = U.seqlen - U.q_len + U.i0 + U.nrows - 1;
       for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
-        const int st = it % kIdxStages;
-        if (!warp_wait(smem_u32(&kempty[st]), ((it / kIdxStages) & 1) ^ 1, TO, abort_flag)) {
+        const int st = it % kS;
+        if (!warp_wait(smem_u32(&kempty[st]), ((it / kS) & 1) ^ 1, TO, abort_flag)) {
           ok = false;
           break;
         }
@@ -437,16 +449,17 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
       }
     }
     cp_async_wait_all();
-  } else if (warp < 4) {
+  } else if (kLean ? warp == 2 : warp < 4) {
     // ------------------------------------------------------------ query quantizers
-    const int qw = warp - 2;  // 0..1
+    const int qw = warp - 2;  // 0..1 (the lean form has warp 2 only)
+    constexpr int kQW = kLean ? 1 : 2;  // quantizer warps
     uint32_t un = 0;
     IdxCursor cur{sh.gs, sh.ts};
     IdxUnit U;
     while (!*abort_flag && idx_next(p, sh, cur, U)) {
       const int qb = un & 1;
       if (!warp_wait(smem_u32(&qempty[qb]), ((un >> 1) & 1) ^ 1, TO, abort_flag)) break;
-      uint8_t* qdst = qbuf + qb * kIdxQBufBytes;
+      uint8_t* qdst = qbuf + qb * kQB;
       float* wdst = wq + qb * 4 * kIdxHeads;
       // A half-warp converts one 128-element row (8 elements = 16 B per lane);
       // kQRows rows per half-warp are loaded before any is used, so their
@@ -454,12 +467,12 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
       // stream, so each round trip is long). Rows r = base + 4 i of the batch.
       constexpr int kQRows = 16;
       const int half = lane >> 4, hl = lane & 15;
-      for (int base = qw * 2 + half; base < N; base += 4 * kQRows) {
+      for (int base = qw * 2 + half; base < N; base += 2 * kQW * kQRows) {
         uint4 raw[kQRows];
         float wj[kQRows];
 #pragma unroll
         for (int i = 0; i < kQRows; ++i) {
-          const int r = base + 4 * i;
+          const int r = base + 2 * kQW * i;
           const int gi = r / kIdxHeads, j = r % kIdxHeads;
           raw[i] = make_uint4(0u, 0u, 0u, 0u);
           wj[i] = 0.f;
@@ -472,7 +485,7 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
         }
 #pragma unroll
         for (int i = 0; i < kQRows; ++i) {
-          const int r = base + 4 * i;  // < N: N is a multiple of 64
+          const int r = base + 2 * kQW * i;  // < N: N is a multiple of 64
           const uint32_t wv[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
           float x[8];
 #pragma unroll
@@ -501,10 +514,11 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int wg = (warp - 4) >> 2;    // warpgroup: owns TMEM accumulator `wg`
+    const int wg = kLean ? 0 : (warp - 4) >> 2;  // warpgroup: takes every other tile
     const int quad = warp & 3;         // TMEM lane quadrant of this warp
     const int e = quad * 32 + lane;    // key within the tile == TMEM lane
-    const int et = tid - 4 * 32;       // 0..255 among the epilogue threads
+    const int et = tid - 4 * 32;       // 0..255 among the epilogue threads (filter mode)
+    constexpr int kNext = kLean ? 1 : 2;  // this warpgroup's next tile
     int cpar = 0;                      // filter mode: staging buffer of the next tile
     uint32_t it = 0, un = 0;
     if (blockIdx.x == 0 && wg == 0) {  // sequences whose rows or length are out of range
@@ -563,15 +577,15 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
       };
       bool ok = true;
       for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
-        if ((int)(it & 1) != wg) continue;  // the other warpgroup's tile
+        if (!kLean && (int)(it & 1) != wg) continue;  // the other warpgroup's tile
         const int s = kt * p.tile_stride * kIdxTile + e;  // this thread's key
         const float ks = pf_kt == kt ? pf_ks : scale_of(kt);
-        if (kt + 2 < U.kt1) {
-          pf_ks = scale_of(kt + 2);
-          pf_kt = kt + 2;
+        if (kt + kNext < U.kt1) {
+          pf_ks = scale_of(kt + kNext);
+          pf_kt = kt + kNext;
         }
         const int ab = (int)(it % (uint32_t)nacc);  // accumulator of this tile
-        if (!warp_wait(smem_u32(&kempty[it % kIdxStages]), (it / kIdxStages) & 1, TO, abort_flag)) {
+        if (!warp_wait(smem_u32(&kempty[it % kS]), (it / kS) & 1, TO, abort_flag)) {
           ok = false;
           break;
         }
@@ -591,8 +605,8 @@ __global__ void __launch_bounds__(kAssist ? kIdxAssistThreads : kIdxThreads, 1)
             cstage[((cpar * 4 + gi) << 8) + et] = score_key(out);
           }
         };
-        if constexpr (kAssist) {
-          // 16-column chunks (the 16-warp form's register budget): row gi's 64 head
+        if constexpr (kAssist || kLean) {
+          // 16-column chunks (the 16-warp and two-CTA forms' register budget): row gi's 64 head
           // columns as four chunks, the next one's load in flight while one is reduced
           uint32_t ca[16], cb[16];
           tmem_ld16u(tcol, ca);
