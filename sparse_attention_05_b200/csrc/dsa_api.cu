@@ -15,9 +15,6 @@
 #include "../../include/dsa.h"
 #include "ptx.cuh"
 #include "topk.cuh"
-#ifndef DSA_IDX_LEAN
-#define DSA_IDX_LEAN 1
-#endif
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
 #include "indexer_kl.cuh"
@@ -259,7 +256,6 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
                             int row_begin, int row_count, cudaStream_t stream,
                             int tile_stride = 1, const IdxFilter& filt = IdxFilter()) {
   static DeviceOnce once;
-  constexpr bool kIdxLeanDecode = DSA_IDX_LEAN;
   const cudaError_t attr_err = once_per_device(once, [] {
     cudaError_t e = cudaFuncSetAttribute(indexer_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmemBytes);
@@ -268,9 +264,6 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
                                kIdxSmemBytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(indexer_kernel<false, true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(indexer_kernel<false, false, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kIdxLeanSmemBytes);
     return e;
   });
@@ -315,13 +308,10 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   const int grid = (int)std::min<int64_t>(max_tiles, num_sms());
   if (p.thr) {
     indexer_kernel<true><<<grid, kIdxThreads, kIdxSmemBytes, stream>>>(p, tm);
-  } else if (kIdxLeanDecode && p.G <= 2) {
-    // decode groups: two lean CTAs per SM
+  } else if (p.G <= 2) {
+    // decode groups: two lean CTAs per SM (each takes an equal share as well)
     const int grid2 = (int)std::min<int64_t>(max_tiles, 2 * (int64_t)num_sms());
-    indexer_kernel<false, false, true><<<grid2, kIdxLeanThreads, kIdxLeanSmemBytes, stream>>>(p, tm);
-  } else if (p.paged && p.G <= 2) {
-    // paged decode: the copy warps take half of each tile's 8-KB random-page reads
-    indexer_kernel<false, true><<<grid, kIdxAssistThreads, kIdxSmemBytes, stream>>>(p, tm);
+    indexer_kernel<false, true><<<grid2, kIdxLeanThreads, kIdxLeanSmemBytes, stream>>>(p, tm);
   } else {
     indexer_kernel<false><<<grid, kIdxThreads, kIdxSmemBytes, stream>>>(p, tm);
   }

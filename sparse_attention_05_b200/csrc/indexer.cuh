@@ -31,6 +31,9 @@
 // A stage of the ring carries key codes only and is reused as soon as the MMA has
 // read it (the scales never gate a stage); the same commit tells the epilogue that
 // the tile's accumulator is ready.
+// Decode groups (G <= 2) run a lean form instead: two CTAs per SM, each with warps 0-2
+// as above (one quantizer warp), warps 3-6 a single epilogue warpgroup, 4 key stages
+// and 256 TMEM columns, so two tile pipelines share each SM.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -45,11 +48,6 @@ constexpr int kIdxDim = 128;
 constexpr int kIdxTile = 128;                      // keys per tile (MMA M)
 constexpr int kIdxStages = 8;
 constexpr int kIdxThreads = 384;
-// Paged decode form: four more warps (12-15) bring the second half of every key tile
-// with cp.async beside the producer's TMA box (see indexer_kernel's kAssist).
-constexpr int kIdxAssistThreads = 512;
-constexpr int kIdxCpWarp0 = 12;
-constexpr int kIdxCpThreads = 128;
 constexpr int kIdxStageBytes = kIdxTile * kIdxDim;  // 16 KB of e4m3
 constexpr int kIdxQBufBytes = 4 * kIdxHeads * kIdxDim;  // G <= 4 rows x 64 heads x 128 B
 constexpr int kIdxSmemBytes =
@@ -68,7 +66,7 @@ constexpr int kIdxLeanSmemBytes = 1024 + kIdxLeanStages * kIdxStageBytes +
 
 struct IndexerParams {
   const __nv_bfloat16* q_idx;  // [T][64][128]
-  const uint8_t* k_idx;        // [cache_rows][128] E4M3 key codes (the copy warps' half tiles)
+  const uint8_t* k_idx;        // [cache_rows][128] E4M3 key codes
   int64_t cache_rows;
   const float* w;              // [T][64]
   const float* k_scale;        // [cache_rows]
@@ -225,20 +223,15 @@ __device__ void idx_share(const IndexerParams& p, IdxShare* out, uint32_t* scrat
 
 // kFilter: the fused selection's filter mode (thr, cand_* set; no score rows); the
 // plain instantiation carries none of its code.
-// kAssist (paged caches, at most 2 query rows per group): each key tile arrives as one
-// TMA box of 64 keys (the producer) and 64 keys copied in 16-B cp.async pieces by four
-// extra warps. A per-SM trace of the paged decode showed the producer's TMA issue
-// holding only about two tiles in flight (one 8-KB random-page box per ~800 cycles),
-// so the tile stream was bound by the TMA unit; the copy warps take half of it. The
-// 16 warps leave 128 registers per thread, so the epilogue reads tensor memory in
-// 16-column chunks.
-template <bool kFilter, bool kAssist = false, bool kLean = false>
-__global__ void __launch_bounds__(kLean ? kIdxLeanThreads : (kAssist ? kIdxAssistThreads : kIdxThreads),
-                                  kLean ? 2 : 1)
+// kLean (groups of at most 2 query rows, i.e. decode): two CTAs per SM with 7 warps
+// each (warps 3-6 one epilogue warpgroup that takes every tile), 4 key stages and 256
+// TMEM columns; 2 x 224 threads leave 144 registers per thread, so the epilogue reads
+// tensor memory in 16-column chunks.
+template <bool kFilter, bool kLean = false>
+__global__ void __launch_bounds__(kLean ? kIdxLeanThreads : kIdxThreads, kLean ? 2 : 1)
     indexer_kernel(const __grid_constant__ IndexerParams p,
                    const __grid_constant__ CUtensorMap tm_keys) {
-  static_assert(!(kFilter && kAssist), "the copy-assisted form is for plain scores");
-  static_assert(!(kLean && (kFilter || kAssist)), "the lean form is for plain scores");
+  static_assert(!(kLean && kFilter), "the lean form is for plain scores");
   constexpr int kS = kLean ? kIdxLeanStages : kIdxStages;        // key stages
   constexpr int kQB = kLean ? kIdxLeanQBufBytes : kIdxQBufBytes;  // one query buffer
   extern __shared__ uint8_t smem_raw[];
@@ -277,7 +270,7 @@ __global__ void __launch_bounds__(kLean ? kIdxLeanThreads : (kAssist ? kIdxAssis
   if (tid == 0) {
     for (int s = 0; s < kS; ++s) {
       // expect_tx arrival (+ the TMA bytes), and one arrival per copy thread
-      mbar_init(smem_u32(&kfull[s]), kAssist ? 1 + kIdxCpThreads : 1);
+      mbar_init(smem_u32(&kfull[s]), 1);  // the producer's expect_tx arrival (+ TMA bytes)
       mbar_init(smem_u32(&kempty[s]), 1);  // the MMA's commit (stage free, scores ready)
     }
     for (int i = 0; i < kIdxMaxAcc; ++i) mbar_init(smem_u32(&tempty[i]), 128);
@@ -351,9 +344,9 @@ __global__ void __launch_bounds__(kLean ? kIdxLeanThreads : (kAssist ? kIdxAssis
           }
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(bar, kAssist ? kIdxStageBytes / 2 : kIdxStageBytes);
+          mbar_arrive_expect_tx(bar, kIdxStageBytes);
 #pragma unroll
-          for (int h = 0; h < (kAssist ? 1 : 2); ++h)  // kAssist: keys 64-127 by the copy warps
+          for (int h = 0; h < 2; ++h)
             tma_load_2d(smem_u32(stages + st * kIdxStageBytes + h * 8192), &tm_keys, bar, 0,
                         (int)base[h]);
         }
@@ -385,7 +378,6 @@ __global__ void __launch_bounds__(kLean ? kIdxLeanThreads : (kAssist ? kIdxAssis
             break;
           }
           tc_fence_after();
-          if (kAssist) fence_proxy_async_smem();  // cp.async (generic proxy) -> tensor core
           const uint32_t kaddr = smem_u32(stages + st * kIdxStageBytes);
           const uint32_t dcol = tmem_base + ab * N;
 #pragma unroll
@@ -405,50 +397,6 @@ __global__ void __launch_bounds__(kLean ? kIdxLeanThreads : (kAssist ? kIdxAssis
       mbar_wait(smem_u32(mdone), 0, TO, no_abort);
     }
     __syncwarp();
-  } else if (kAssist && warp >= kIdxCpWarp0) {
-    // ------------------------------------------------------------ cp.async copy warps
-    // Keys 64-127 of each tile (64 rows x 128 B) in 16-B pieces, four per thread,
-    // written in the 128-B swizzled layout the TMA gives the first half; each thread
-    // arrives on the stage barrier once its pieces have landed. Rows past the cache
-    // end (a contiguous cache whose length is not a multiple of 128) read as zeros.
-    const int ct = tid - kIdxCpWarp0 * 32;
-    uint32_t it = 0;
-    IdxCursor cur{sh.gs, sh.ts};
-    IdxUnit U;
-    bool ok = true;
-    while (ok && !*abort_flag && idx_next(p, sh, cur, U)) {
-      const int pos_max = U.seqlen - U.q_len + U.i0 + U.nrows - 1;
-      for (int kt = U.kt0; kt < U.kt1; ++kt, ++it) {
-        const int st = it % kS;
-        if (!warp_wait(smem_u32(&kempty[st]), ((it / kS) & 1) ^ 1, TO, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const int s0 = kt * p.tile_stride * kIdxTile + 64;
-        int64_t base = 0;  // past pos_max or behind a bad page: row 0 (masked later)
-        if (s0 <= pos_max) {
-          if (!p.paged) {
-            base = (int64_t)U.b * p.max_ctx + s0;
-          } else {
-            const int page = __ldg(p.block_table + (int64_t)U.b * p.max_pages + s0 / p.page_size);
-            if (page >= 0 && page < p.num_pages)
-              base = (int64_t)page * p.page_size + s0 % p.page_size;
-          }
-        }
-        const uint8_t* src = p.k_idx + base * kIdxDim;
-        const uint32_t dst = smem_u32(stages + st * kIdxStageBytes + 8192);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = ct + kIdxCpThreads * i;  // piece: row c / 8, 16-B column c % 8
-          const int r = c >> 3, j = c & 7;
-          const bool in = base + r < p.cache_rows;
-          cp_async_16(dst + r * 128 + ((j ^ (r & 7)) << 4), in ? src + r * 128 + j * 16 : p.k_idx,
-                      in ? 16u : 0u);
-        }
-        cp_async_mbar_arrive(smem_u32(&kfull[st]));
-      }
-    }
-    cp_async_wait_all();
   } else if (kLean ? warp == 2 : warp < 4) {
     // ------------------------------------------------------------ query quantizers
     const int qw = warp - 2;  // 0..1 (the lean form has warp 2 only)
@@ -605,8 +553,8 @@ __global__ void __launch_bounds__(kLean ? kIdxLeanThreads : (kAssist ? kIdxAssis
             cstage[((cpar * 4 + gi) << 8) + et] = score_key(out);
           }
         };
-        if constexpr (kAssist || kLean) {
-          // 16-column chunks (the 16-warp and two-CTA forms' register budget): row gi's 64 head
+        if constexpr (kLean) {
+          // 16-column chunks (the two-CTA form's register budget): row gi's 64 head
           // columns as four chunks, the next one's load in flight while one is reduced
           uint32_t ca[16], cb[16];
           tmem_ld16u(tcol, ca);
